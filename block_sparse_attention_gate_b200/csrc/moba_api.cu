@@ -1,0 +1,335 @@
+// C ABI of the MoBA causal-prefill library: argument validation, workspace carve-up and
+// the launch sequence (pool -> gate -> route -> block attention + merge).  Nothing here
+// allocates or synchronises; every kernel is enqueued on the caller's stream.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "moba.h"
+#include "moba_internal.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+void set_err(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
+moba_status fail(moba_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+moba_status cuda_fail(cudaError_t e, const char* where) {
+  set_err("%s: %s", where, cudaGetErrorString(e));
+  return MOBA_ERR_CUDA;
+}
+
+constexpr int64_t kI32Max = 2147483647LL;
+
+// Validate the parameters and derive the kernels' geometry (host only).
+moba_status make_geom(const moba_params* p, moba::Geom* g) {
+  if (!p) return fail(MOBA_ERR_INVALID_ARG, "params is NULL");
+  if (p->num_seqs < 1) return fail(MOBA_ERR_INVALID_ARG, "num_seqs must be >= 1 (got %d)", p->num_seqs);
+  if (p->num_seqs > 65535) return fail(MOBA_ERR_UNSUPPORTED, "num_seqs must be <= 65535 (got %d)", p->num_seqs);
+  if (p->num_q_heads < 1 || p->num_kv_heads < 1 || p->num_q_heads % p->num_kv_heads)
+    return fail(MOBA_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)",
+                p->num_q_heads, p->num_kv_heads);
+  if (p->head_dim != 64 && p->head_dim != 128)
+    return fail(MOBA_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", p->head_dim);
+  if (p->block_size < 128 || p->block_size % 128 || p->block_size > 8192)
+    return fail(MOBA_ERR_UNSUPPORTED, "block_size must be a multiple of 128 in [128, 8192] (got %d)",
+                p->block_size);
+  if (p->top_k < 1 || p->top_k > moba::kMaxTopK)
+    return fail(MOBA_ERR_UNSUPPORTED, "top_k must be in [1, %d] (got %d)", moba::kMaxTopK, p->top_k);
+  if ((int64_t)p->num_kv_heads * p->head_dim > 16384)
+    return fail(MOBA_ERR_UNSUPPORTED, "num_kv_heads * head_dim must be <= 16384");
+  int64_t T = 0, maxlen = 0;
+  if (p->cu_seqlens_host) {
+    if (!p->cu_seqlens) return fail(MOBA_ERR_INVALID_ARG, "cu_seqlens (device) is NULL but the host copy is not");
+    if (p->cu_seqlens_host[0] != 0) return fail(MOBA_ERR_INVALID_ARG, "cu_seqlens[0] must be 0");
+    for (int s = 0; s < p->num_seqs; ++s) {
+      int64_t len = (int64_t)p->cu_seqlens_host[s + 1] - p->cu_seqlens_host[s];
+      if (len < 0) return fail(MOBA_ERR_INVALID_ARG, "cu_seqlens must be nondecreasing (at %d)", s);
+      if (len > maxlen) maxlen = len;
+    }
+    T = p->cu_seqlens_host[p->num_seqs];
+    if (((uintptr_t)p->cu_seqlens) & 3) return fail(MOBA_ERR_ALIGNMENT, "cu_seqlens (device) misaligned");
+  } else {
+    if (p->cu_seqlens) return fail(MOBA_ERR_INVALID_ARG, "cu_seqlens given without cu_seqlens_host");
+    if (p->max_seqlen < 0) return fail(MOBA_ERR_INVALID_ARG, "max_seqlen must be >= 0");
+    maxlen = p->max_seqlen;
+    T = (int64_t)p->num_seqs * maxlen;
+  }
+  if (T > kI32Max) return fail(MOBA_ERR_UNSUPPORTED, "total tokens exceed 2^31-1");
+  const int64_t MB = (maxlen + p->block_size - 1) / p->block_size;
+  if (MB > 16384) return fail(MOBA_ERR_UNSUPPORTED, "more than 16384 blocks in one sequence");
+  if (T * p->num_q_heads * p->top_k > kI32Max)
+    return fail(MOBA_ERR_UNSUPPORTED, "T * Hq * top_k exceeds 2^31-1");
+  g->cu = p->cu_seqlens_host ? p->cu_seqlens : nullptr;
+  g->num_seqs = p->num_seqs;
+  g->L = (int32_t)(p->cu_seqlens_host ? 0 : maxlen);
+  g->T = (int32_t)T;
+  g->Hq = p->num_q_heads;
+  g->Hkv = p->num_kv_heads;
+  g->G = p->num_q_heads / p->num_kv_heads;
+  g->D = p->head_dim;
+  g->bs = p->block_size;
+  g->MB = (int32_t)MB;
+  g->k = p->top_k;
+  g->scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf((float)p->head_dim);
+  g->scale_log2 = g->scale * 1.4426950408889634f;
+  g->nbk = (int64_t)p->num_kv_heads * p->num_seqs * MB;
+  g->R = T * p->num_q_heads * (p->top_k - 1);
+  return MOBA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace carve-up; with base == nullptr only the size is computed.
+size_t carve(const moba::Geom& g, char* base, moba::Work* w) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* ptr = base ? base + off : nullptr;
+    off += align256(bytes);
+    return ptr;
+  };
+  moba::Work x;
+  x.counts = (int32_t*)take(sizeof(int32_t) * (size_t)g.nbk);
+  x.offsets = (int32_t*)take(sizeof(int32_t) * (size_t)(g.nbk + 1));
+  x.cursors = (int32_t*)take(sizeof(int32_t) * (size_t)g.nbk);
+  x.tile_off = (int32_t*)take(sizeof(int32_t) * (size_t)(g.nbk + 1));
+  x.rows = (int32_t*)take(sizeof(int32_t) * (size_t)g.R);
+  x.part_o = (float*)take(sizeof(float) * (size_t)g.R * g.D);
+  x.part_lse = (float*)take(sizeof(float) * (size_t)g.R);
+  x.kbar = (float*)take(sizeof(float) * (size_t)g.num_seqs * g.MB * g.Hkv * g.D);
+  x.sel = (int32_t*)take(sizeof(int32_t) * (size_t)g.T * g.Hq * g.k);
+  x.bytes = off;
+  if (w) *w = x;
+  return off;
+}
+
+moba_status check_device() {
+  int dev = 0, major = 0, minor = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  if (major != 10 || minor != 0)
+    return fail(MOBA_ERR_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a", dev, major, minor);
+  return MOBA_OK;
+}
+
+bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15) == 0; }
+
+moba_status check_ptr(const void* ptr, const char* name, bool needed) {
+  if (!needed) return MOBA_OK;
+  if (!ptr) return fail(MOBA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(ptr)) return fail(MOBA_ERR_ALIGNMENT, "%s is not 16-byte aligned", name);
+  return MOBA_OK;
+}
+
+moba_status check_ws(const moba::Geom& g, void* ws, size_t bytes, moba::Work* w) {
+  const size_t need = carve(g, nullptr, nullptr);
+  if (need && !ws) return fail(MOBA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+  if (((uintptr_t)ws) & 255) return fail(MOBA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (bytes < need) return fail(MOBA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", bytes, need);
+  carve(g, (char*)ws, w);
+  return MOBA_OK;
+}
+
+#define MOBA_TRY(x)                      \
+  do {                                   \
+    moba_status _s = (x);                \
+    if (_s != MOBA_OK) return _s;        \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t moba_kbar_elems(const moba_params* p) {
+  moba::Geom g;
+  if (make_geom(p, &g) != MOBA_OK) return 0;
+  return (size_t)g.num_seqs * g.MB * g.Hkv * g.D;
+}
+
+size_t moba_workspace_size(const moba_params* p) {
+  moba::Geom g;
+  if (make_geom(p, &g) != MOBA_OK) return 0;
+  return carve(g, nullptr, nullptr);
+}
+
+moba_status moba_pool_keys(const moba_params* p, const void* K, float* Kbar, void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0 || g.MB == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(K, "K", true));
+  MOBA_TRY(check_ptr(Kbar, "Kbar", true));
+  MOBA_TRY(check_device());
+  cudaError_t e = moba::launch_pool(g, (const __nv_bfloat16*)K, Kbar, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOBA_OK : cuda_fail(e, "pool launch");
+}
+
+moba_status moba_gate_topk(const moba_params* p, const void* Q, const float* Kbar, int32_t* sel,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(Q, "Q", true));
+  MOBA_TRY(check_ptr(Kbar, "Kbar", true));
+  MOBA_TRY(check_ptr(sel, "sel", true));
+  moba::Work w;
+  MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
+  MOBA_TRY(check_device());
+  cudaError_t e = moba::launch_gate(g, (const __nv_bfloat16*)Q, Kbar, sel, w, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOBA_OK : cuda_fail(e, "gate launch");
+}
+
+static moba_status attn_stages(const moba::Geom& g, const void* Q, const void* K, const void* V,
+                               const int32_t* sel, const moba::Work& w, void* O, float* LSE,
+                               cudaStream_t st, int which /* 1 route, 2 past, 4 self */) {
+  cudaError_t e = cudaSuccess;
+  if ((which & 1) && g.k > 1) {
+    e = moba::launch_route(g, sel, w, st);
+    if (e != cudaSuccess) return cuda_fail(e, "route launch");
+  }
+  if (which & 2) {
+    e = moba::launch_attn_past(g, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, w, st);
+    if (e != cudaSuccess) return cuda_fail(e, "past-block attention launch");
+  }
+  if (which & 4) {
+    e = moba::launch_attn_self(g, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, sel,
+                               w, (__nv_bfloat16*)O, LSE, st);
+    if (e != cudaSuccess) return cuda_fail(e, "own-block attention launch");
+  }
+  return MOBA_OK;
+}
+
+moba_status moba_attn_fwd(const moba_params* p, const void* Q, const void* K, const void* V,
+                          const int32_t* sel, void* workspace, size_t workspace_bytes, void* O,
+                          float* LSE, void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(Q, "Q", true));
+  MOBA_TRY(check_ptr(K, "K", true));
+  MOBA_TRY(check_ptr(V, "V", true));
+  MOBA_TRY(check_ptr(sel, "sel", true));
+  MOBA_TRY(check_ptr(O, "O", true));
+  MOBA_TRY(check_ptr(LSE, "LSE", true));
+  moba::Work w;
+  MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
+  MOBA_TRY(check_device());
+  return attn_stages(g, Q, K, V, sel, w, O, LSE, (cudaStream_t)stream, 7);
+}
+
+moba_status moba_route(const moba_params* p, const int32_t* sel, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(sel, "sel", true));
+  moba::Work w;
+  MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
+  MOBA_TRY(check_device());
+  return attn_stages(g, nullptr, nullptr, nullptr, sel, w, nullptr, nullptr, (cudaStream_t)stream, 1);
+}
+
+moba_status moba_attn_past(const moba_params* p, const void* Q, const void* K, const void* V, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(Q, "Q", true));
+  MOBA_TRY(check_ptr(K, "K", true));
+  MOBA_TRY(check_ptr(V, "V", true));
+  moba::Work w;
+  MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
+  MOBA_TRY(check_device());
+  return attn_stages(g, Q, K, V, nullptr, w, nullptr, nullptr, (cudaStream_t)stream, 2);
+}
+
+moba_status moba_attn_self_merge(const moba_params* p, const void* Q, const void* K, const void* V,
+                                 const int32_t* sel, void* workspace, size_t workspace_bytes, void* O,
+                                 float* LSE, void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(Q, "Q", true));
+  MOBA_TRY(check_ptr(K, "K", true));
+  MOBA_TRY(check_ptr(V, "V", true));
+  MOBA_TRY(check_ptr(sel, "sel", true));
+  MOBA_TRY(check_ptr(O, "O", true));
+  MOBA_TRY(check_ptr(LSE, "LSE", true));
+  moba::Work w;
+  MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
+  MOBA_TRY(check_device());
+  return attn_stages(g, Q, K, V, sel, w, O, LSE, (cudaStream_t)stream, 4);
+}
+
+int moba_launches_per_forward(const moba_params* p) {
+  moba::Geom g;
+  if (make_geom(p, &g) != MOBA_OK) return -1;
+  if (g.T == 0) return 0;
+  return moba::launches_per_forward(g);
+}
+
+moba_status moba_fwd(const moba_params* p, const void* Q, const void* K, const void* V, float* Kbar,
+                     int32_t* sel, void* workspace, size_t workspace_bytes, void* O, float* LSE,
+                     void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(Q, "Q", true));
+  MOBA_TRY(check_ptr(K, "K", true));
+  MOBA_TRY(check_ptr(V, "V", true));
+  MOBA_TRY(check_ptr(O, "O", true));
+  MOBA_TRY(check_ptr(LSE, "LSE", true));
+  MOBA_TRY(check_ptr(Kbar, "Kbar", Kbar != nullptr));
+  MOBA_TRY(check_ptr(sel, "sel", sel != nullptr));
+  moba::Work w;
+  MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
+  MOBA_TRY(check_device());
+  float* kb = Kbar ? Kbar : w.kbar;
+  int32_t* sl = sel ? sel : w.sel;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = moba::launch_pool(g, (const __nv_bfloat16*)K, kb, st);
+  if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+  e = moba::launch_gate(g, (const __nv_bfloat16*)Q, kb, sl, w, st);
+  if (e != cudaSuccess) return cuda_fail(e, "gate launch");
+  return attn_stages(g, Q, K, V, sl, w, O, LSE, st, 7);
+}
+
+const char* moba_status_string(int status) {
+  switch (status) {
+    case MOBA_OK: return "ok";
+    case MOBA_ERR_INVALID_ARG: return "invalid argument";
+    case MOBA_ERR_UNSUPPORTED: return "unsupported size";
+    case MOBA_ERR_ALIGNMENT: return "misaligned pointer";
+    case MOBA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOBA_ERR_CUDA: return "CUDA error";
+    case MOBA_ERR_DEVICE: return "unsupported device";
+    default: return "unknown status";
+  }
+}
+
+const char* moba_last_error(void) { return g_err; }
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// Internal definitions shared by the MoBA kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace moba {
+
+constexpr int kMaxTopK = 16;
+
+// Problem geometry as the kernels see it (passed by value).
+struct Geom {
+  const int32_t* cu;  // device offsets, or nullptr for uniform sequences of length L
+  int32_t num_seqs;
+  int32_t L;          // uniform sequence length (cu == nullptr)
+  int32_t T;          // total tokens
+  int32_t Hq, Hkv, G, D;
+  int32_t bs;         // block size
+  int32_t MB;         // max blocks per sequence
+  int32_t k;          // top_k (own block included)
+  float scale;        // softmax scale
+  float scale_log2;   // softmax scale * log2(e)
+  int64_t nbk;        // routing buckets: Hkv * num_seqs * MB
+  int64_t R;          // routed partial rows: T * Hq * (k - 1)
+};
+
+__device__ __forceinline__ int32_t seq_start(const Geom& g, int s) {
+  return g.cu ? __ldg(g.cu + s) : s * g.L;
+}
+__device__ __forceinline__ int32_t seq_end(const Geom& g, int s) {
+  return g.cu ? __ldg(g.cu + s + 1) : (s + 1) * g.L;
+}
+// Sequence holding token t (binary search over the offsets).
+__device__ __forceinline__ int find_seq(const Geom& g, int32_t t) {
+  if (!g.cu) return t / g.L;
+  int lo = 0, hi = g.num_seqs - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(g.cu + mid) <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Workspace carve-up (device pointers; every region 256-byte aligned).
+struct Work {
+  int32_t* counts;    // [nbk] rows routed to each (kv head, sequence, block) bucket
+  int32_t* offsets;   // [nbk + 1] exclusive scan of counts
+  int32_t* cursors;   // [nbk] scatter cursors
+  int32_t* tile_off;  // [nbk + 1] exclusive scan of per-bucket tile counts
+  int32_t* rows;      // [R] routed partial ids, grouped by bucket
+  float* part_o;      // [R, D] normalised partial outputs
+  float* part_lse;    // [R] partial log-sum-exp
+  float* kbar;        // [num_seqs, MB, Hkv, D] (used by moba_fwd when the caller passes none)
+  int32_t* sel;       // [T, Hq, k] (used by moba_fwd when the caller passes none)
+  size_t bytes;       // total
+};
+
+// Launchers (each returns the launch's cudaError_t).
+cudaError_t launch_pool(const Geom& g, const __nv_bfloat16* K, float* Kbar, cudaStream_t st);
+cudaError_t launch_gate(const Geom& g, const __nv_bfloat16* Q, const float* Kbar, int32_t* sel,
+                        const Work& w, cudaStream_t st);
+cudaError_t launch_route(const Geom& g, const int32_t* sel, const Work& w, cudaStream_t st);
+cudaError_t launch_attn_past(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                             const __nv_bfloat16* V, const Work& w, cudaStream_t st);
+cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                             const __nv_bfloat16* V, const int32_t* sel, const Work& w,
+                             __nv_bfloat16* O, float* LSE, cudaStream_t st);
+// Number of kernel launches one forward pass enqueues (pool, gate, route, attention).
+int launches_per_forward(const Geom& g);
+
+}  // namespace moba

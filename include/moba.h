@@ -1,0 +1,163 @@
+/*
+ * moba.h -- C ABI of the MoBA (Mixture of Block Attention) causal-prefill library
+ * for NVIDIA B200 (sm_100a).
+ *
+ * MoBA splits the keys of every sequence into equal blocks, mean-pools each
+ * block's keys, lets every query score the pooled keys of its past blocks with a
+ * parameter-free dot product, keeps its own block plus the best-scoring past
+ * blocks (top_k in all), runs exact softmax attention over the chosen blocks only
+ * (causal inside its own block) and merges the per-block results by online
+ * softmax.  Sources: the MoBA project README ("MoBA: Mixture of Block Attention for
+ * Long-Context LLMs", gittoolsai.com mirror: "Trainable Block Sparse Attention",
+ * "Parameter-less Gating Mechanism", FAQ of GitHub issue #27), and the youleyou.com
+ * article "Kimi发布MoBA突破性实现无限上下文" (sections "MoBA：基于块的混合注意力机制"
+ * and "PyTorch实现关键要点").
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller, 16-byte aligned,
+ *    contiguous, row-major.  Q is [T, Hq, D] bf16; K and V are [T, Hkv, D] bf16;
+ *    T = total tokens of the packed batch (varlen packing by cu_seqlens).
+ *  - The library never allocates, never synchronises the host, and enqueues its
+ *    kernels asynchronously on `stream` (a cudaStream_t passed as void*; NULL is the
+ *    legacy default stream).  Scratch comes from the caller's `workspace`.
+ *  - Argument errors are reported before anything is enqueued.  A failed launch
+ *    returns MOBA_ERR_CUDA; moba_last_error() then holds a message (per thread).
+ *  - Block b of sequence s covers tokens [cu[s] + b*bs, min(cu[s] + (b+1)*bs, cu[s+1])).
+ *    Block indices in `sel` are local to the sequence.
+ *  - Kbar is laid out [num_seqs, MB, Hkv, D] fp32 with MB = ceil(max_seqlen / bs)
+ *    (blocks past a sequence's end are written as zeros).
+ *  - LSE is the natural-log log-sum-exp of the scaled logits, fp32 [T, Hq].
+ */
+#ifndef MOBA_H_
+#define MOBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOBA_API __attribute__((visibility("default")))
+#else
+#define MOBA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOBA_OK = 0,
+  MOBA_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent cu_seqlens */
+  MOBA_ERR_UNSUPPORTED = 2, /* a size the kernels do not handle (head_dim, block_size, top_k) */
+  MOBA_ERR_ALIGNMENT = 3,   /* a device pointer is not 16-byte aligned */
+  MOBA_ERR_WORKSPACE = 4,   /* workspace missing, too small or not 256-byte aligned */
+  MOBA_ERR_CUDA = 5,        /* a CUDA runtime call or a kernel launch failed */
+  MOBA_ERR_DEVICE = 6       /* the current device is not an sm_100 (B200-class) GPU */
+} moba_status;
+
+typedef struct {
+  int32_t num_seqs;               /* >= 1 */
+  const int32_t* cu_seqlens_host; /* HOST, num_seqs+1 offsets, [0] = 0, nondecreasing;
+                                     NULL: num_seqs sequences of max_seqlen tokens each */
+  const int32_t* cu_seqlens;      /* DEVICE copy of the same offsets (NULL iff the host copy is) */
+  int32_t max_seqlen;             /* used only when cu_seqlens_host is NULL */
+  int32_t num_q_heads;            /* Hq, a multiple of num_kv_heads (GQA group G = Hq/Hkv) */
+  int32_t num_kv_heads;           /* Hkv */
+  int32_t head_dim;               /* D: 64 or 128 */
+  int32_t block_size;             /* bs: a multiple of 128, at most 8192 */
+  int32_t top_k;                  /* blocks per query including its own block: 1..16 */
+  float softmax_scale;            /* <= 0 means 1/sqrt(head_dim) */
+} moba_params;
+
+/* Number of fp32 elements of Kbar: num_seqs * MB * Hkv * D (0 if params are invalid). */
+MOBA_API size_t moba_kbar_elems(const moba_params* p);
+
+/* Bytes of workspace that moba_gate_topk, moba_attn_fwd and moba_fwd need (host only,
+ * no CUDA call).  Returns 0 if params are invalid. */
+MOBA_API size_t moba_workspace_size(const moba_params* p);
+
+/*
+ * Block mean-pooling of the keys (each block's representative is the mean of its
+ * keys; youleyou.com article, section "MoBA：基于块的混合注意力机制", and its
+ * implementation section "PyTorch实现关键要点").
+ *   K     [T, Hkv, D] bf16, read once.
+ *   Kbar  [num_seqs, MB, Hkv, D] fp32 out: mean over the block's valid tokens,
+ *         accumulated in fp32.
+ */
+MOBA_API moba_status moba_pool_keys(const moba_params* p, const void* K, float* Kbar, void* stream);
+
+/*
+ * Parameter-free gate with causal block mask, forced own block and top-k (README
+ * bullet "Parameter-less Gating Mechanism"; README FAQ of issue #27: the own block
+ * is always taken, top_k-1 more come from strictly earlier blocks, the own block is
+ * not a candidate; the article's section "PyTorch实现关键要点": score = query times
+ * pooled key, mask future blocks, top-k).
+ *   Q     [T, Hq, D] bf16.
+ *   Kbar  from moba_pool_keys.
+ *   sel   [T, Hq, top_k] int32 out: sel[..,0] = own block i = floor(p/bs);
+ *         sel[..,1..m] = the m = min(top_k-1, i) past blocks with the largest
+ *         <q, Kbar[b]>, by descending score, ties to the lower block index;
+ *         remaining slots -1.
+ *   workspace: >= moba_workspace_size(p) bytes, 256-byte aligned.
+ */
+MOBA_API moba_status moba_gate_topk(const moba_params* p, const void* Q, const float* Kbar, int32_t* sel,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Attention over the selected blocks plus online-softmax merge (article section
+ * "PyTorch实现关键要点": attention runs separately on the own block, causally, and on
+ * the chosen blocks, and the partial results are merged by online softmax; README
+ * FAQ of issue #27: the own block goes through the causal varlen path).
+ *   Q, K, V  as above; sel from moba_gate_topk (or any caller-made selection that
+ *            obeys its contract: slot 0 the own block, then distinct past blocks,
+ *            -1 padding at the end).
+ *   O    [T, Hq, D] bf16 out;  LSE  [T, Hq] fp32 out.
+ *   Scales logits by softmax_scale (default 1/sqrt(D)); fp32 accumulation.
+ */
+MOBA_API moba_status moba_attn_fwd(const moba_params* p, const void* Q, const void* K, const void* V,
+                          const int32_t* sel, void* workspace, size_t workspace_bytes, void* O,
+                          float* LSE, void* stream);
+
+/*
+ * The whole forward pass: pool, gate, attention.  Kbar and sel may be NULL, in
+ * which case they live inside the workspace; when given they receive the
+ * intermediate results (same layouts as above).
+ */
+MOBA_API moba_status moba_fwd(const moba_params* p, const void* Q, const void* K, const void* V,
+                     float* Kbar, int32_t* sel, void* workspace, size_t workspace_bytes, void* O,
+                     float* LSE, void* stream);
+
+/*
+ * Stages of moba_attn_fwd, callable one by one (moba_attn_fwd = route, past, own
+ * block + merge, in this order, on one stream; the workspace carries the state).
+ *   moba_route:           groups every (token, query head, slot >= 1) by the past
+ *                         block it selected (per KV head), MoE-style: counts, scans,
+ *                         scatter (article section "PyTorch实现关键要点": organise the
+ *                         data after top-k).  Needs top_k >= 2 to do anything.
+ *   moba_attn_past:       exact softmax attention of every routed query row over the
+ *                         whole selected block (a past block is complete and wholly
+ *                         visible); writes normalised partials + LSE into the workspace.
+ *   moba_attn_self_merge: causal attention inside each query's own block, then the
+ *                         online-softmax merge with the partials; writes O and LSE.
+ */
+MOBA_API moba_status moba_route(const moba_params* p, const int32_t* sel, void* workspace,
+                                size_t workspace_bytes, void* stream);
+MOBA_API moba_status moba_attn_past(const moba_params* p, const void* Q, const void* K, const void* V,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+MOBA_API moba_status moba_attn_self_merge(const moba_params* p, const void* Q, const void* K,
+                                          const void* V, const int32_t* sel, void* workspace,
+                                          size_t workspace_bytes, void* O, float* LSE, void* stream);
+
+/* Kernel launches one moba_fwd enqueues for these params (host only; -1 if invalid). */
+MOBA_API int moba_launches_per_forward(const moba_params* p);
+
+/* Static description of a status code. */
+MOBA_API const char* moba_status_string(int status);
+
+/* Detail of the last error raised on the calling thread ("" if none). */
+MOBA_API const char* moba_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOBA_H_ */
