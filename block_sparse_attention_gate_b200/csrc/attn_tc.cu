@@ -1,0 +1,447 @@
+// MoBA block attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Two modes share one kernel body:
+//   past : a CTA takes a tile of up to 128 routed query rows of one bucket (KV head g,
+//          sequence s, past block b), attends the whole block (bs keys; a past block is
+//          complete and fully visible) and writes normalised fp32 partials + LSE.
+//   own  : a CTA takes 128 consecutive tokens of one query head inside one block, attends
+//          the block's keys up to the diagonal (causal mask on the diagonal chunk), then
+//          merges the past partials of every row by online softmax and writes O (bf16) and
+//          LSE.
+// (youleyou.com, "Kimi发布MoBA突破性实现无限上下文", section "PyTorch实现关键要点": attention
+// runs on the own block and on the selected blocks separately and the results are merged by
+// online softmax; zhuoshang.net, "MoBA是什么？…", section "MoBA的技术原理": causal mask inside
+// the current block.)
+//
+// Per 128-key chunk j:  S_j = Q K_j^T  (tcgen05, fp32 in TMEM, double-buffered)
+//                       softmax rows in registers (one thread per row), P_j -> smem (bf16)
+//                       O += P_j V_j    (tcgen05, fp32 accumulator in TMEM)
+// Warp roles: warps 0-3 softmax + epilogue (thread r owns row r = TMEM lane r), warp 4 TMA
+// producer (K/V chunks, two stages), warp 5 TMEM owner + MMA issuer.
+#include <cudaTypedefs.h>
+#include <float.h>
+
+#include "moba_internal.cuh"
+#include "sm100.cuh"
+
+namespace moba {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kRows = 128;  // query rows per CTA (M)
+constexpr int kBN = 128;    // keys per chunk (N of S, K of PV)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColO = 256;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct AttnArgs {
+  Geom g;
+  const __nv_bfloat16* Q;
+  const int32_t* sel;
+  const int32_t* offsets;
+  const int32_t* tile_off;
+  const int32_t* rows;
+  float* part_o;
+  float* part_lse;
+  __nv_bfloat16* O;
+  float* LSE;
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kTile = kRows * D * 2;  // bytes of a [128 x D] bf16 tile
+  static constexpr int kQ = 0;
+  static constexpr int kK0 = kQ + kTile;
+  static constexpr int kV0 = kK0 + 2 * kTile;
+  static constexpr int kP = kV0 + 2 * kTile;
+  static constexpr int kBar = kP + kRows * kBN * 2;
+  static constexpr int kBytes = kBar + 256;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+};
+
+enum Bar { kQFull = 0, kKVFull0, kKVFull1, kKVEmpty0, kKVEmpty1, kSFull0, kSFull1, kSFree0, kSFree1, kPFull, kPVDone, kDone, kNumBars };
+
+template <int D, bool kOwn>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kNumBars * 8);
+  const Geom& g = a.g;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ------------------------------------------------------------- work item
+  int gk, h = 0, s;
+  int32_t key0, nrows, row_start = 0, q0 = 0, i_blk = 0;
+  int nchunks;
+  if constexpr (!kOwn) {
+    const int32_t total = __ldg(a.tile_off + g.nbk);
+    const int32_t tile = (int32_t)blockIdx.x;
+    if (tile >= total) return;
+    int64_t lo = 0, hi = g.nbk - 1;  // last bucket whose first tile is <= tile
+    while (lo < hi) {
+      const int64_t mid = (lo + hi + 1) >> 1;
+      if (__ldg(a.tile_off + mid) <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int32_t b = (int32_t)(lo % g.MB);
+    s = (int)((lo / g.MB) % g.num_seqs);
+    gk = (int)(lo / ((int64_t)g.MB * g.num_seqs));
+    row_start = __ldg(a.offsets + lo) + (tile - __ldg(a.tile_off + lo)) * kRows;
+    nrows = min(kRows, __ldg(a.offsets + lo + 1) - row_start);
+    key0 = seq_start(g, s) + b * g.bs;
+    nchunks = g.bs / kBN;
+  } else {
+    const int per_blk = g.bs / kRows;
+    i_blk = blockIdx.x / per_blk;
+    const int qt = blockIdx.x - i_blk * per_blk;
+    s = blockIdx.y;
+    h = blockIdx.z;
+    gk = h / g.G;
+    const int32_t ts = seq_start(g, s), te = seq_end(g, s);
+    key0 = ts + i_blk * g.bs;
+    q0 = key0 + qt * kRows;
+    if (q0 >= te) return;
+    nrows = min(kRows, te - q0);
+    nchunks = qt + 1;
+  }
+
+  // ------------------------------------------------------------- setup
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (tid == 0) {
+    mbar_init(&bars[kQFull], kRows);
+    mbar_init(&bars[kKVFull0], 1);
+    mbar_init(&bars[kKVFull1], 1);
+    mbar_init(&bars[kKVEmpty0], 1);
+    mbar_init(&bars[kKVEmpty1], 1);
+    mbar_init(&bars[kSFull0], 1);
+    mbar_init(&bars[kSFull1], 1);
+    mbar_init(&bars[kSFree0], kRows);
+    mbar_init(&bars[kSFree1], kRows);
+    mbar_init(&bars[kPFull], kRows);
+    mbar_init(&bars[kPVDone], 1);
+    mbar_init(&bars[kDone], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sQ = smem_u32(smem + L::kQ);
+  const uint32_t sK0 = smem_u32(smem + L::kK0);
+  const uint32_t sV0 = smem_u32(smem + L::kV0);
+  const uint32_t sP = smem_u32(smem + L::kP);
+  bool ok = true;
+
+  if (warp < 4) {
+    // ========================================================= softmax warps
+    const int r = tid;
+    int64_t qrow = -1;
+    int32_t e = -1;
+    if (r < nrows) {
+      if constexpr (!kOwn) {
+        e = __ldg(a.rows + row_start + r);
+        qrow = e / (g.k - 1);
+      } else {
+        qrow = (int64_t)(q0 + r) * g.Hq + h;
+      }
+    }
+    {  // gather this row of Q into the swizzled tile (zeros for padding rows)
+      const __nv_bfloat16* src = qrow >= 0 ? a.Q + qrow * D : a.Q;
+      const uint32_t nb = qrow >= 0 ? 16u : 0u;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) cp_async_16(sQ + sw128_offset(r, c, kRows), src + c * 8, nb);
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[kQFull]);
+    }
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float c2 = g.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    for (int j = 0; j < nchunks && ok; ++j) {
+      const int sb = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull0 + sb], (j >> 1) & 1, g.err));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + kColS0 + sb * kBN + c * 32, sr[c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars[kSFree0 + sb]);
+      const bool diag = kOwn && (j == nchunks - 1);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          float v = __uint_as_float(sr[c][x]) * c2;
+          if (diag && (c * 32 + x) > r) v = -INFINITY;
+          sr[c][x] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      const float m_new = fmaxf(m, mx);
+      const float alpha = ex2(m - m_new);
+      float rs = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const float p0 = ex2(__uint_as_float(sr[c][x]) - m_new);
+          const float p1 = ex2(__uint_as_float(sr[c][x + 1]) - m_new);
+          rs += p0 + p1;
+          pk[(c * 32 + x) >> 1] = pack_bf16x2(p0, p1);
+        }
+      l = l * alpha + rs;
+      m = m_new;
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kPVDone], (j - 1) & 1, g.err));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_off + kColO + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+            tmem_st32(tmem + lane_off + kColO + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      uint8_t* pbase = smem + L::kP;
+#pragma unroll
+      for (int c16 = 0; c16 < kBN / 8; ++c16) {
+        uint4 v = make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+        *reinterpret_cast<uint4*>(pbase + sw128_offset(r, c16, kRows)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars[kPFull]);
+    }
+    // ------------------------------------------------------- epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kPVDone], (nchunks - 1) & 1, g.err));
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const float lse_row = (m + __log2f(l)) * kLn2;
+      if constexpr (!kOwn) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + kColO + c * 32, o);
+          tmem_wait_ld();
+          if (r < nrows) {
+            float4* dst = reinterpret_cast<float4*>(a.part_o + (int64_t)e * D + c * 32);
+#pragma unroll
+            for (int x = 0; x < 32; x += 4)
+              dst[x >> 2] = make_float4(__uint_as_float(o[x]) * inv_l, __uint_as_float(o[x + 1]) * inv_l,
+                                        __uint_as_float(o[x + 2]) * inv_l, __uint_as_float(o[x + 3]) * inv_l);
+          }
+        }
+        if (r < nrows) a.part_lse[e] = lse_row;
+      } else {
+        // online-softmax merge of the own-block result with the row's past partials
+        float M = lse_row;
+        int32_t pe[kMaxTopK];
+        float pl[kMaxTopK];
+        int np = 0;
+        if (r < nrows) {
+          for (int slot = 1; slot < g.k; ++slot) {
+            const int32_t b = __ldg(a.sel + qrow * g.k + slot);
+            if (b >= 0 && b < i_blk) {
+              pe[np] = (int32_t)(qrow * (g.k - 1) + slot - 1);
+              pl[np] = __ldg(a.part_lse + pe[np]);
+              M = fmaxf(M, pl[np]);
+              ++np;
+            }
+          }
+        }
+        const float w_self = __expf(lse_row - M);
+        float sumw = w_self;
+        for (int q = 0; q < np; ++q) {
+          pl[q] = __expf(pl[q] - M);
+          sumw += pl[q];
+        }
+        const float inv_w = 1.f / sumw;
+        const float a_self = w_self * inv_l * inv_w;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + kColO + c * 32, o);
+          tmem_wait_ld();
+          if (r < nrows) {
+            float acc[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) acc[x] = __uint_as_float(o[x]) * a_self;
+            for (int q = 0; q < np; ++q) {
+              const float4* src = reinterpret_cast<const float4*>(a.part_o + (int64_t)pe[q] * D + c * 32);
+              const float wq = pl[q] * inv_w;
+#pragma unroll
+              for (int x = 0; x < 32; x += 4) {
+                const float4 v = __ldg(src + (x >> 2));
+                acc[x] = fmaf(wq, v.x, acc[x]);
+                acc[x + 1] = fmaf(wq, v.y, acc[x + 1]);
+                acc[x + 2] = fmaf(wq, v.z, acc[x + 2]);
+                acc[x + 3] = fmaf(wq, v.w, acc[x + 3]);
+              }
+            }
+            uint4* dst = reinterpret_cast<uint4*>(a.O + qrow * D + c * 32);
+#pragma unroll
+            for (int x = 0; x < 32; x += 8)
+              dst[x >> 3] = make_uint4(pack_bf16x2(acc[x], acc[x + 1]), pack_bf16x2(acc[x + 2], acc[x + 3]),
+                                       pack_bf16x2(acc[x + 4], acc[x + 5]), pack_bf16x2(acc[x + 6], acc[x + 7]));
+          }
+        }
+        if (r < nrows) a.LSE[qrow] = M + __logf(sumw);
+      }
+    }
+  } else if (warp == 4) {
+    // ========================================================= TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      for (int j = 0; j < nchunks && ok; ++j) {
+        const int st = j & 1, u = j >> 1;
+        if (u > 0) {
+          ok = mbar_wait(&bars[kKVEmpty0 + st], (u - 1) & 1, g.err);
+          if (!ok) break;
+        }
+        uint64_t* full = &bars[kKVFull0 + st];
+        mbar_expect_tx(full, 2u * L::kTile);
+        const int t = key0 + j * kBN;
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh) {
+          tma_load_3d(smem + L::kK0 + st * L::kTile + hh * kRows * 128, &tmK, full, hh * 64, gk, t);
+          tma_load_3d(smem + L::kV0 + st * L::kTile + hh * kRows * 128, &tmV, full, hh * 64, gk, t);
+        }
+      }
+    }
+  } else {
+    // ========================================================= MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(kRows, kBN, false, false);
+      constexpr uint32_t idO = idesc_bf16(kRows, D, false, true);
+      auto issue_pv = [&](int c) -> bool {
+        if (!mbar_wait(&bars[kPFull], c & 1, g.err)) return false;
+        tc_fence_after();
+        const uint32_t vb = sV0 + (c & 1) * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(sP + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(vb + kk * 2048, kRows * 128, 1024);
+          mma_bf16_ss(tmem + kColO, ad, bd, idO, (c > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars[kPVDone]);
+        mma_commit(&bars[kKVEmpty0 + (c & 1)]);
+        return true;
+      };
+      ok = mbar_wait(&bars[kQFull], 0, g.err);
+      for (int j = 0; j < nchunks && ok; ++j) {
+        const int st = j & 1, sb = j & 1;
+        ok = mbar_wait(&bars[kKVFull0 + st], (j >> 1) & 1, g.err);
+        if (ok && j >= 2) ok = mbar_wait(&bars[kSFree0 + sb], ((j >> 1) - 1) & 1, g.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb = sK0 + st * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(kb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
+          mma_bf16_ss(tmem + kColS0 + sb * kBN, ad, bd, idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[kSFull0 + sb]);
+        if (j >= 1) ok = issue_pv(j - 1);
+      }
+      if (ok) ok = issue_pv(nchunks - 1);
+      // every MMA issued above has completed once kDone fires
+      mma_commit(&bars[kDone]);
+      mbar_wait(&bars[kDone], 0, g.err);
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [T, Hkv, D] bf16 viewed as dims (d, kv head, token); boxes of 64 d x 1 head x 128 tokens,
+// 128-byte swizzle (the canonical K-major / MN-major atoms of the MMA operands).
+cudaError_t make_kv_map(CUtensorMap* m, const void* base, const Geom& g) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.Hkv, (cuuint64_t)g.T};
+  const cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.Hkv * g.D * 2};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)kBN};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D, bool kOwn>
+cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                      const int32_t* sel, const Work& w, __nv_bfloat16* O, float* LSE, dim3 grid, cudaStream_t st) {
+  CUtensorMap tk, tv;
+  cudaError_t e = make_kv_map(&tk, K, g);
+  if (e != cudaSuccess) return e;
+  e = make_kv_map(&tv, V, g);
+  if (e != cudaSuccess) return e;
+  AttnArgs a{g, Q, sel, w.offsets, w.tile_off, w.rows, w.part_o, w.part_lse, O, LSE};
+  const int smem = Layout<D>::kAlloc;
+  e = cudaFuncSetAttribute(attn_tc_kernel<D, kOwn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<D, kOwn><<<grid, kThreads, smem, st>>>(tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_past(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                             const __nv_bfloat16* V, const Work& w, cudaStream_t st) {
+  if (g.T == 0 || g.k < 2 || g.R == 0) return cudaSuccess;
+  const int64_t tiles = (g.R + kRows - 1) / kRows + g.nbk;  // upper bound of the routed tile count
+  dim3 grid((unsigned)tiles);
+  if (g.D == 64) return launch_tc<64, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, grid, st);
+  return launch_tc<128, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, grid, st);
+}
+
+cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                             const __nv_bfloat16* V, const int32_t* sel, const Work& w,
+                             __nv_bfloat16* O, float* LSE, cudaStream_t st) {
+  if (g.T == 0) return cudaSuccess;
+  dim3 grid((unsigned)(g.MB * (g.bs / kRows)), (unsigned)g.num_seqs, (unsigned)g.Hq);
+  if (g.D == 64) return launch_tc<64, true>(g, Q, K, V, sel, w, O, LSE, grid, st);
+  return launch_tc<128, true>(g, Q, K, V, sel, w, O, LSE, grid, st);
+}
+
+int launches_per_forward(const Geom& g) {
+  // pool + gate + (route count, scan, scatter + past attention when top_k > 1) + own block/merge
+  return 2 + (g.k > 1 ? 4 : 0) + 1;
+}
+
+}  // namespace moba

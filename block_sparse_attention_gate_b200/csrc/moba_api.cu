@@ -8,6 +8,9 @@
 #include "moba.h"
 #include "moba_internal.cuh"
 
+// Device error word: kernels OR a code into it when a bounded wait gives up.
+__device__ int g_moba_device_error = 0;
+
 namespace {
 
 thread_local char g_err[512] = "";
@@ -116,7 +119,12 @@ size_t carve(const moba::Geom& g, char* base, moba::Work* w) {
   return off;
 }
 
-moba_status check_device() {
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices] = {};  // device address of g_moba_device_error, per device
+
+// Checks that the current device is an sm_100 part and binds the device error word's
+// address (looked up once per device with that device current) into the geometry.
+moba_status check_device(moba::Geom* g) {
   int dev = 0, major = 0, minor = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -126,6 +134,14 @@ moba_status check_device() {
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
   if (major != 10 || minor != 0)
     return fail(MOBA_ERR_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a", dev, major, minor);
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOBA_ERR_DEVICE, "device ordinal %d out of range", dev);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_moba_device_error);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  g->err = g_err_ptr[dev];
   return MOBA_OK;
 }
 
@@ -176,7 +192,7 @@ moba_status moba_pool_keys(const moba_params* p, const void* K, float* Kbar, voi
   if (g.T == 0 || g.MB == 0) return MOBA_OK;
   MOBA_TRY(check_ptr(K, "K", true));
   MOBA_TRY(check_ptr(Kbar, "Kbar", true));
-  MOBA_TRY(check_device());
+  MOBA_TRY(check_device(&g));
   cudaError_t e = moba::launch_pool(g, (const __nv_bfloat16*)K, Kbar, (cudaStream_t)stream);
   return e == cudaSuccess ? MOBA_OK : cuda_fail(e, "pool launch");
 }
@@ -192,7 +208,7 @@ moba_status moba_gate_topk(const moba_params* p, const void* Q, const float* Kba
   MOBA_TRY(check_ptr(sel, "sel", true));
   moba::Work w;
   MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
-  MOBA_TRY(check_device());
+  MOBA_TRY(check_device(&g));
   cudaError_t e = moba::launch_gate(g, (const __nv_bfloat16*)Q, Kbar, sel, w, (cudaStream_t)stream);
   return e == cudaSuccess ? MOBA_OK : cuda_fail(e, "gate launch");
 }
@@ -232,7 +248,7 @@ moba_status moba_attn_fwd(const moba_params* p, const void* Q, const void* K, co
   MOBA_TRY(check_ptr(LSE, "LSE", true));
   moba::Work w;
   MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
-  MOBA_TRY(check_device());
+  MOBA_TRY(check_device(&g));
   return attn_stages(g, Q, K, V, sel, w, O, LSE, (cudaStream_t)stream, 7);
 }
 
@@ -245,7 +261,7 @@ moba_status moba_route(const moba_params* p, const int32_t* sel, void* workspace
   MOBA_TRY(check_ptr(sel, "sel", true));
   moba::Work w;
   MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
-  MOBA_TRY(check_device());
+  MOBA_TRY(check_device(&g));
   return attn_stages(g, nullptr, nullptr, nullptr, sel, w, nullptr, nullptr, (cudaStream_t)stream, 1);
 }
 
@@ -260,7 +276,7 @@ moba_status moba_attn_past(const moba_params* p, const void* Q, const void* K, c
   MOBA_TRY(check_ptr(V, "V", true));
   moba::Work w;
   MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
-  MOBA_TRY(check_device());
+  MOBA_TRY(check_device(&g));
   return attn_stages(g, Q, K, V, nullptr, w, nullptr, nullptr, (cudaStream_t)stream, 2);
 }
 
@@ -279,7 +295,7 @@ moba_status moba_attn_self_merge(const moba_params* p, const void* Q, const void
   MOBA_TRY(check_ptr(LSE, "LSE", true));
   moba::Work w;
   MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
-  MOBA_TRY(check_device());
+  MOBA_TRY(check_device(&g));
   return attn_stages(g, Q, K, V, sel, w, O, LSE, (cudaStream_t)stream, 4);
 }
 
@@ -306,7 +322,7 @@ moba_status moba_fwd(const moba_params* p, const void* Q, const void* K, const v
   MOBA_TRY(check_ptr(sel, "sel", sel != nullptr));
   moba::Work w;
   MOBA_TRY(check_ws(g, workspace, workspace_bytes, &w));
-  MOBA_TRY(check_device());
+  MOBA_TRY(check_device(&g));
   float* kb = Kbar ? Kbar : w.kbar;
   int32_t* sl = sel ? sel : w.sel;
   cudaStream_t st = (cudaStream_t)stream;
@@ -331,5 +347,21 @@ const char* moba_status_string(int status) {
 }
 
 const char* moba_last_error(void) { return g_err; }
+
+moba_status moba_read_device_error(int32_t* value, int clear) {
+  g_err[0] = 0;
+  if (!value) return fail(MOBA_ERR_INVALID_ARG, "value is NULL");
+  moba::Geom g;
+  MOBA_TRY(check_device(&g));
+  int v = 0;
+  cudaError_t e = cudaMemcpy(&v, g.err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (clear) {
+    e = cudaMemset(g.err, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  }
+  *value = v;
+  return MOBA_OK;
+}
 
 }  // extern "C"

@@ -23,6 +23,7 @@ struct Geom {
   float scale_log2;   // softmax scale * log2(e)
   int64_t nbk;        // routing buckets: Hkv * num_seqs * MB
   int64_t R;          // routed partial rows: T * Hq * (k - 1)
+  int* err;           // device error word (bounded waits that gave up), never null
 };
 
 __device__ __forceinline__ int32_t seq_start(const Geom& g, int s) {

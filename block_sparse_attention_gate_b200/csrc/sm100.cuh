@@ -9,9 +9,6 @@
 
 namespace moba {
 
-// Set (never cleared by the kernels) when a bounded wait gives up; read by moba_device_error().
-extern __device__ int g_moba_device_error;
-
 // ~2 s at 2 GHz: no legitimate wait in these kernels comes close
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
@@ -47,14 +44,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete.  Gives up after kWaitLimitCycles,
-// records the failure in g_moba_device_error and returns false (the caller then skips its
-// remaining work and goes to teardown).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// ORs kErrWaitTimeout into *err (the library's device error word) and returns false; the
+// caller then skips its remaining work and goes to teardown.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > kWaitLimitCycles) {
-      atomicOr(&g_moba_device_error, kErrWaitTimeout);
+      atomicOr(err, kErrWaitTimeout);
       return false;
     }
   }

@@ -150,6 +150,14 @@ MOBA_API moba_status moba_attn_self_merge(const moba_params* p, const void* Q, c
 /* Kernel launches one moba_fwd enqueues for these params (host only; -1 if invalid). */
 MOBA_API int moba_launches_per_forward(const moba_params* p);
 
+/*
+ * Device error word of the current device: the tensor-core kernels bound every wait on an
+ * mbarrier (about 2 s); a wait that gives up ORs 1 into this word and the kernel returns
+ * early instead of hanging.  Reads it synchronously (and zeroes it when `clear` != 0).
+ * A non-zero value means the outputs of the affected launches are not valid.
+ */
+MOBA_API moba_status moba_read_device_error(int32_t* value, int clear);
+
 /* Static description of a status code. */
 MOBA_API const char* moba_status_string(int status);
 

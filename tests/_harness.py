@@ -59,6 +59,7 @@ def run_gpu(w: synth.Workload, Q: np.ndarray, K: np.ndarray, V: np.ndarray, stag
     else:
         mb.moba_fwd(p, Qd, Kd, Vd, ws, O, LSE, Kbar=kbar, sel=sel)
     torch.cuda.synchronize()
+    assert mb.moba_read_device_error(clear=True) == 0, "a kernel wait gave up"
     return {
         "Kbar": kbar.view(w.num_seqs, p.max_blocks, w.num_kv_heads, D).cpu().numpy(),
         "sel": sel.cpu().numpy(),
