@@ -376,40 +376,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// [T, Hkv, D] bf16 viewed as dims (d, kv head, token); boxes of 64 d x 1 head x 128 tokens,
-// 128-byte swizzle (the canonical K-major / MN-major atoms of the MMA operands).
-cudaError_t make_kv_map(CUtensorMap* m, const void* base, const Geom& g) {
-  auto fn = encode_fn();
-  if (!fn) return cudaErrorNotSupported;
-  const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.Hkv, (cuuint64_t)g.T};
-  const cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.Hkv * g.D * 2};
-  const cuuint32_t box[3] = {64, 1, (cuuint32_t)kBN};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 template <int D, bool kOwn>
 cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                       const int32_t* sel, const Work& w, __nv_bfloat16* O, float* LSE, dim3 grid, cudaStream_t st) {
   CUtensorMap tk, tv;
-  cudaError_t e = make_kv_map(&tk, K, g);
+  cudaError_t e = make_rows_map(&tk, K, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
-  e = make_kv_map(&tv, V, g);
+  e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
   AttnArgs a{g, Q, sel, w.offsets, w.tile_off, w.rows, w.part_o, w.part_lse, O, LSE};
   const int smem = Layout<D>::kAlloc;
@@ -440,8 +413,39 @@ cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_b
 }
 
 int launches_per_forward(const Geom& g) {
-  // pool + gate + (route count, scan, scatter + past attention when top_k > 1) + own block/merge
-  return 2 + (g.k > 1 ? 4 : 0) + 1;
+  // pool + gate (Kbar split, scores/top-k) + (route count, scan, scatter + past attention
+  // when top_k > 1) + own block/merge
+  return 3 + (g.k > 1 ? 4 : 0) + 1;
+}
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+}  // namespace
+
+// A [rows, heads, D] bf16 tensor viewed as dims (d, head, row); boxes of 64 d x 1 head x
+// box_rows rows with the 128-byte swizzle, i.e. the canonical 128-byte-swizzled atoms of the
+// MMA operands (K-major for Q, K, Kbar; MN-major for V).  Out-of-range rows read as zeros.
+cudaError_t make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, int heads, int D, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 }  // namespace moba

@@ -1,0 +1,266 @@
+// Parameter-free MoBA gate on the tensor cores: scores s = <q, Kbar[b]> for the strictly
+// earlier blocks of the query's sequence, forced own block, top-(k-1) past blocks by
+// descending score with ties to the lower block index.  (MoBA README, "Parameter-less
+// Gating Mechanism" and the FAQ answer of GitHub issue #27: the own block is always taken
+// and is not a candidate, k-1 more blocks come from earlier blocks; youleyou.com,
+// "Kimi发布MoBA突破性实现无限上下文", section "PyTorch实现关键要点": score by the product of the
+// query with the pooled keys, mask future blocks, top-k.)
+//
+// A CTA takes 128 consecutive tokens of one query head inside one query block i.  The
+// candidate blocks 0..i-1 are processed in chunks of up to 128: the chunk's pooled keys,
+// split into bf16 hi + lo parts (Kbar = hi + lo + O(2^-17 |Kbar|)), are staged by TMA and
+// S = Q hi^T + Q lo^T accumulates in fp32 TMEM (double-buffered).  Thread r reads row r
+// of S from TMEM and keeps a sorted running top-(k-1) list in registers.
+#include <cudaTypedefs.h>
+#include <float.h>
+
+#include "moba_internal.cuh"
+#include "sm100.cuh"
+
+namespace moba {
+
+
+namespace {
+
+constexpr int kThreads = 160;     // warps 0-3 epilogue, warp 4 TMA + MMA
+constexpr int kRows = 128;        // query rows per CTA
+constexpr int kCand = 128;        // candidate blocks per chunk
+constexpr int kBoxRows = 64;      // candidate rows per TMA box
+constexpr uint32_t kTmemCols = 256;
+constexpr int kMaxM = kMaxTopK - 1;
+
+template <int D>
+struct GLayout {
+  static constexpr int kQ = 0;                       // [128 x D] bf16
+  static constexpr int kHi = kQ + kRows * D * 2;     // [128 x D] bf16
+  static constexpr int kLo = kHi + kCand * D * 2;    // [128 x D] bf16
+  static constexpr int kBar = kLo + kCand * D * 2;
+  static constexpr int kAlloc = kBar + 128 + 1024;
+};
+
+enum GBar { kFull = 0, kKFree, kTFull0, kTFull1, kTFree0, kTFree1, kGDone, kGNumBars };
+
+__device__ __forceinline__ bool ranks_before(float sa, int32_t ba, float sb, int32_t bb) {
+  return sa > sb || (sa == sb && ba < bb);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+    gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmHi,
+                   const __grid_constant__ CUtensorMap tmLo, Geom g, int32_t* __restrict__ sel) {
+  using L = GLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kGNumBars * 8);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  const int per_blk = g.bs / kRows;
+  const int i = blockIdx.x / per_blk;  // query block (local to the sequence)
+  const int qt = blockIdx.x - i * per_blk;
+  const int s = blockIdx.y, h = blockIdx.z, gk = h / g.G;
+  const int32_t ts = seq_start(g, s), te = seq_end(g, s);
+  const int32_t q0 = ts + i * g.bs + qt * kRows;
+  if (q0 >= te) return;
+  const int nrows = min(kRows, te - q0);
+  const int m = min(g.k - 1, i);  // past blocks to choose
+  if (m == 0) {  // nothing to score: own block only
+    for (int r = tid; r < nrows; r += kThreads) {
+      int32_t* out = sel + ((int64_t)(q0 + r) * g.Hq + h) * g.k;
+      out[0] = i;
+      for (int q = 1; q < g.k; ++q) out[q] = -1;
+    }
+    return;
+  }
+  const int nch = (i + kCand - 1) / kCand;
+
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (tid == 0) {
+    mbar_init(&bars[kFull], 1);
+    mbar_init(&bars[kKFree], 1);
+    mbar_init(&bars[kTFull0], 1);
+    mbar_init(&bars[kTFull1], 1);
+    mbar_init(&bars[kTFree0], kRows);
+    mbar_init(&bars[kTFree1], kRows);
+    mbar_init(&bars[kGDone], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t kb_row0 = (int64_t)s * g.MB;  // first pooled-key row of this sequence
+  bool ok = true;
+
+  if (warp < 4) {
+    // ========================================================= epilogue: running top-m
+    const int r = tid;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    float ts_[kMaxM];
+    int32_t tb_[kMaxM];
+#pragma unroll
+    for (int q = 0; q < kMaxM; ++q) {
+      ts_[q] = -FLT_MAX;
+      tb_[q] = INT32_MAX;
+    }
+    float thr = -FLT_MAX;
+    int32_t thr_b = INT32_MAX;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int buf = c & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kTFull0 + buf], (c >> 1) & 1, g.err));
+      if (!ok) break;
+      tc_fence_after();
+      const int c0 = c * kCand;
+      const int ncand = min(kCand, i - c0);
+      for (int x0 = 0; x0 < ncand; x0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + buf * kCand + x0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const int32_t b = c0 + x0 + x;
+          float sc = __uint_as_float(v[x]);
+          if (b < i && ranks_before(sc, b, thr, thr_b)) {
+            int32_t cb = b;
+#pragma unroll
+            for (int q = 0; q < kMaxM; ++q) {
+              if (q < m && ranks_before(sc, cb, ts_[q], tb_[q])) {
+                const float t1 = ts_[q];
+                const int32_t t2 = tb_[q];
+                ts_[q] = sc;
+                tb_[q] = cb;
+                sc = t1;
+                cb = t2;
+              }
+            }
+#pragma unroll
+            for (int q = 0; q < kMaxM; ++q)
+              if (q == m - 1) {
+                thr = ts_[q];
+                thr_b = tb_[q];
+              }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[kTFree0 + buf]);
+    }
+    if (ok && r < nrows) {
+      int32_t* out = sel + ((int64_t)(q0 + r) * g.Hq + h) * g.k;
+      out[0] = i;
+#pragma unroll
+      for (int q = 0; q < kMaxM; ++q)
+        if (q < m) out[1 + q] = tb_[q];
+      for (int q = 1 + m; q < g.k; ++q) out[q] = -1;
+    }
+  } else if (lane == 0) {
+    // ========================================================= TMA + MMA issuer
+    auto load_chunk = [&](int c, bool with_q) {
+      const int c0 = c * kCand;
+      const int ncand = min(kCand, i - c0);
+      const int nbox = (ncand + kBoxRows - 1) / kBoxRows;
+      uint32_t bytes = (uint32_t)nbox * kBoxRows * D * 2 * 2;
+      if (with_q) bytes += kRows * D * 2;
+      mbar_expect_tx(&bars[kFull], bytes);
+      if (with_q)
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_3d(smem + L::kQ + hh * kRows * 128, &tmQ, &bars[kFull], hh * 64, h, q0);
+      for (int bx = 0; bx < nbox; ++bx)
+        for (int hh = 0; hh < D / 64; ++hh) {
+          const int row = (int)(kb_row0 + c0 + bx * kBoxRows);
+          const int off = hh * kCand * 128 + bx * kBoxRows * 128;
+          tma_load_3d(smem + L::kHi + off, &tmHi, &bars[kFull], hh * 64, gk, row);
+          tma_load_3d(smem + L::kLo + off, &tmLo, &bars[kFull], hh * 64, gk, row);
+        }
+    };
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmHi);
+    prefetch_tmap(&tmLo);
+    load_chunk(0, true);
+    const uint32_t sQ = smem_u32(smem + L::kQ);
+    const uint32_t sHi = smem_u32(smem + L::kHi);
+    const uint32_t sLo = smem_u32(smem + L::kLo);
+    for (int c = 0; c < nch && ok; ++c) {
+      const int buf = c & 1;
+      ok = mbar_wait(&bars[kFull], c & 1, g.err);
+      if (ok && c >= 2) ok = mbar_wait(&bars[kTFree0 + buf], ((c >> 1) - 1) & 1, g.err);
+      if (!ok) break;
+      tc_fence_after();
+      const int ncand = min(kCand, i - c * kCand);
+      const int n = (ncand + 15) & ~15;
+      const uint32_t idesc = idesc_bf16(kRows, n, false, false);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+        const uint32_t boff = (kk >> 2) * (kCand * 128) + (kk & 3) * 32;
+        const uint64_t ad = sdesc_sw128(sQ + koff, 16, 1024);
+        mma_bf16_ss(tmem + buf * kCand, ad, sdesc_sw128(sHi + boff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        mma_bf16_ss(tmem + buf * kCand, ad, sdesc_sw128(sLo + boff, 16, 1024), idesc, 1u);
+      }
+      mma_commit(&bars[kTFull0 + buf]);
+      if (c + 1 < nch) {
+        mma_commit(&bars[kKFree]);
+        ok = mbar_wait(&bars[kKFree], c & 1, g.err);
+        if (!ok) break;
+        load_chunk(c + 1, false);
+      }
+    }
+    mma_commit(&bars[kGDone]);
+    mbar_wait(&bars[kGDone], 0, g.err);
+  }
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Kbar (fp32) -> bf16 hi = rn(x), lo = rn(x - hi).
+__global__ void kbar_split_kernel(const float* __restrict__ kbar, __nv_bfloat16* __restrict__ hi,
+                                  __nv_bfloat16* __restrict__ lo, int64_t n) {
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
+    const float x = kbar[idx];
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    hi[idx] = h;
+    lo[idx] = __float2bfloat16_rn(x - __bfloat162float(h));
+  }
+}
+
+template <int D>
+cudaError_t launch_gate_d(const Geom& g, const __nv_bfloat16* Q, int32_t* sel, const Work& w, cudaStream_t st) {
+  CUtensorMap tq, th, tl;
+  cudaError_t e = make_rows_map(&tq, Q, (uint64_t)g.T, g.Hq, D, kRows);
+  if (e != cudaSuccess) return e;
+  const uint64_t nb = (uint64_t)g.num_seqs * g.MB;
+  e = make_rows_map(&th, w.kbar_hi, nb, g.Hkv, D, kBoxRows);
+  if (e != cudaSuccess) return e;
+  e = make_rows_map(&tl, w.kbar_lo, nb, g.Hkv, D, kBoxRows);
+  if (e != cudaSuccess) return e;
+  const int smem = GLayout<D>::kAlloc;
+  e = cudaFuncSetAttribute(gate_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)(g.MB * (g.bs / kRows)), (unsigned)g.num_seqs, (unsigned)g.Hq);
+  gate_tc_kernel<D><<<grid, kThreads, smem, st>>>(tq, th, tl, g, sel);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gate(const Geom& g, const __nv_bfloat16* Q, const float* Kbar, int32_t* sel, const Work& w,
+                        cudaStream_t st) {
+  if (g.T == 0) return cudaSuccess;
+  const int64_t n = (int64_t)g.num_seqs * g.MB * g.Hkv * g.D;
+  if (n > 0) {
+    const int64_t want = (n + 255) / 256;
+    const int blocks = (int)(want < 148 * 16 ? want : 148 * 16);
+    kbar_split_kernel<<<blocks, 256, 0, st>>>(Kbar, w.kbar_hi, w.kbar_lo, n);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return g.D == 64 ? launch_gate_d<64>(g, Q, sel, w, st) : launch_gate_d<128>(g, Q, sel, w, st);
+}
+
+}  // namespace moba

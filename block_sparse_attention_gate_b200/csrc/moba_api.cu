@@ -114,6 +114,8 @@ size_t carve(const moba::Geom& g, char* base, moba::Work* w) {
   x.part_lse = (float*)take(sizeof(float) * (size_t)g.R);
   x.kbar = (float*)take(sizeof(float) * (size_t)g.num_seqs * g.MB * g.Hkv * g.D);
   x.sel = (int32_t*)take(sizeof(int32_t) * (size_t)g.T * g.Hq * g.k);
+  x.kbar_hi = (__nv_bfloat16*)take(2 * (size_t)g.num_seqs * g.MB * g.Hkv * g.D);
+  x.kbar_lo = (__nv_bfloat16*)take(2 * (size_t)g.num_seqs * g.MB * g.Hkv * g.D);
   x.bytes = off;
   if (w) *w = x;
   return off;

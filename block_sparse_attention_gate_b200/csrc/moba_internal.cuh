@@ -1,6 +1,7 @@
 // Internal definitions shared by the MoBA kernels and the C-ABI layer.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -53,11 +54,14 @@ struct Work {
   float* part_o;      // [R, D] normalised partial outputs
   float* part_lse;    // [R] partial log-sum-exp
   float* kbar;        // [num_seqs, MB, Hkv, D] (used by moba_fwd when the caller passes none)
+  __nv_bfloat16* kbar_hi;  // [num_seqs, MB, Hkv, D] bf16 rn(Kbar) for the tensor-core gate
+  __nv_bfloat16* kbar_lo;  // [num_seqs, MB, Hkv, D] bf16 rn(Kbar - hi)
   int32_t* sel;       // [T, Hq, k] (used by moba_fwd when the caller passes none)
   size_t bytes;       // total
 };
 
 // Launchers (each returns the launch's cudaError_t).
+cudaError_t make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, int heads, int D, int box_rows);
 cudaError_t launch_pool(const Geom& g, const __nv_bfloat16* K, float* Kbar, cudaStream_t st);
 cudaError_t launch_gate(const Geom& g, const __nv_bfloat16* Q, const float* Kbar, int32_t* sel,
                         const Work& w, cudaStream_t st);
