@@ -27,7 +27,6 @@ constexpr int kRows = 128;        // query rows per CTA
 constexpr int kCand = 128;        // candidate blocks per chunk
 constexpr int kBoxRows = 64;      // candidate rows per TMA box
 constexpr uint32_t kTmemCols = 256;
-constexpr int kMaxM = kMaxTopK - 1;
 
 template <int D>
 struct GLayout {
@@ -44,7 +43,9 @@ __device__ __forceinline__ bool ranks_before(float sa, int32_t ba, float sb, int
   return sa > sb || (sa == sb && ba < bb);
 }
 
-template <int D>
+// kMaxM: compile-time capacity of the running top list (>= top_k - 1), so the list lives
+// in registers and an insertion costs kMaxM compare-and-swap steps.
+template <int D, int kMaxM>
 __global__ void __launch_bounds__(kThreads, 2)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmHi,
                    const __grid_constant__ CUtensorMap tmLo, Geom g, int32_t* __restrict__ sel) {
@@ -99,15 +100,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ========================================================= epilogue: running top-m
     const int r = tid;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // Sorted list (best first) of kMaxM slots; the first kMaxM - m slots hold sentinels that
+    // rank before every score and are never displaced, so the m live slots are the last m
+    // and the current m-th best is always the last slot (no runtime indexing).
     float ts_[kMaxM];
     int32_t tb_[kMaxM];
 #pragma unroll
     for (int q = 0; q < kMaxM; ++q) {
-      ts_[q] = -FLT_MAX;
-      tb_[q] = INT32_MAX;
+      const bool live = q >= kMaxM - m;
+      ts_[q] = live ? -FLT_MAX : FLT_MAX;
+      tb_[q] = live ? INT32_MAX : -1;
     }
-    float thr = -FLT_MAX;
-    int32_t thr_b = INT32_MAX;
     for (int c = 0; c < nch && ok; ++c) {
       const int buf = c & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[kTFull0 + buf], (c >> 1) & 1, g.err));
@@ -123,25 +126,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int x = 0; x < 32; ++x) {
           const int32_t b = c0 + x0 + x;
           float sc = __uint_as_float(v[x]);
-          if (b < i && ranks_before(sc, b, thr, thr_b)) {
+          if (b < i && ranks_before(sc, b, ts_[kMaxM - 1], tb_[kMaxM - 1])) {
             int32_t cb = b;
 #pragma unroll
             for (int q = 0; q < kMaxM; ++q) {
-              if (q < m && ranks_before(sc, cb, ts_[q], tb_[q])) {
-                const float t1 = ts_[q];
-                const int32_t t2 = tb_[q];
-                ts_[q] = sc;
-                tb_[q] = cb;
-                sc = t1;
-                cb = t2;
-              }
+              const bool take = ranks_before(sc, cb, ts_[q], tb_[q]);
+              const float os = ts_[q];
+              const int32_t ob = tb_[q];
+              ts_[q] = take ? sc : os;
+              tb_[q] = take ? cb : ob;
+              sc = take ? os : sc;
+              cb = take ? ob : cb;
             }
-#pragma unroll
-            for (int q = 0; q < kMaxM; ++q)
-              if (q == m - 1) {
-                thr = ts_[q];
-                thr_b = tb_[q];
-              }
           }
         }
       }
@@ -153,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       out[0] = i;
 #pragma unroll
       for (int q = 0; q < kMaxM; ++q)
-        if (q < m) out[1 + q] = tb_[q];
+        if (q >= kMaxM - m) out[1 + q - (kMaxM - m)] = tb_[q];
       for (int q = 1 + m; q < g.k; ++q) out[q] = -1;
     }
   } else if (lane == 0) {
@@ -229,7 +225,7 @@ __global__ void kbar_split_kernel(const float* __restrict__ kbar, __nv_bfloat16*
   }
 }
 
-template <int D>
+template <int D, int kMaxM>
 cudaError_t launch_gate_d(const Geom& g, const __nv_bfloat16* Q, int32_t* sel, const Work& w, cudaStream_t st) {
   CUtensorMap tq, th, tl;
   cudaError_t e = make_rows_map(&tq, Q, (uint64_t)g.T, g.Hq, D, kRows);
@@ -240,10 +236,10 @@ cudaError_t launch_gate_d(const Geom& g, const __nv_bfloat16* Q, int32_t* sel, c
   e = make_rows_map(&tl, w.kbar_lo, nb, g.Hkv, D, kBoxRows);
   if (e != cudaSuccess) return e;
   const int smem = GLayout<D>::kAlloc;
-  e = cudaFuncSetAttribute(gate_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = cudaFuncSetAttribute(gate_tc_kernel<D, kMaxM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(g.MB * (g.bs / kRows)), (unsigned)g.num_seqs, (unsigned)g.Hq);
-  gate_tc_kernel<D><<<grid, kThreads, smem, st>>>(tq, th, tl, g, sel);
+  gate_tc_kernel<D, kMaxM><<<grid, kThreads, smem, st>>>(tq, th, tl, g, sel);
   return cudaGetLastError();
 }
 
@@ -260,7 +256,17 @@ cudaError_t launch_gate(const Geom& g, const __nv_bfloat16* Q, const float* Kbar
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  return g.D == 64 ? launch_gate_d<64>(g, Q, sel, w, st) : launch_gate_d<128>(g, Q, sel, w, st);
+  const int m = g.k - 1;
+  if (g.D == 64) {
+    if (m <= 2) return launch_gate_d<64, 2>(g, Q, sel, w, st);
+    if (m <= 4) return launch_gate_d<64, 4>(g, Q, sel, w, st);
+    if (m <= 8) return launch_gate_d<64, 8>(g, Q, sel, w, st);
+    return launch_gate_d<64, kMaxTopK - 1>(g, Q, sel, w, st);
+  }
+  if (m <= 2) return launch_gate_d<128, 2>(g, Q, sel, w, st);
+  if (m <= 4) return launch_gate_d<128, 4>(g, Q, sel, w, st);
+  if (m <= 8) return launch_gate_d<128, 8>(g, Q, sel, w, st);
+  return launch_gate_d<128, kMaxTopK - 1>(g, Q, sel, w, st);
 }
 
 }  // namespace moba
