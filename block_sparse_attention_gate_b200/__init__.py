@@ -25,7 +25,7 @@ STATUS = {0: "MOBA_OK", 1: "MOBA_ERR_INVALID_ARG", 2: "MOBA_ERR_UNSUPPORTED",
 EXPORTS = ("moba_kbar_elems", "moba_workspace_size", "moba_pool_keys", "moba_gate_topk",
            "moba_attn_fwd", "moba_fwd", "moba_route", "moba_attn_past", "moba_attn_self_merge",
            "moba_launches_per_forward", "moba_read_device_error", "moba_status_string",
-           "moba_last_error")
+           "moba_last_error", "moba_gate_topk_noalloc")
 
 
 class MobaError(RuntimeError):
@@ -71,6 +71,8 @@ def load():
         lib.moba_route.argtypes = [P, vp, vp, sz, vp]
         lib.moba_attn_past.argtypes = [P, vp, vp, vp, vp, sz, vp]
         lib.moba_attn_self_merge.argtypes = [P, vp, vp, vp, vp, vp, sz, vp, vp, vp]
+        lib.moba_gate_topk_noalloc.argtypes = [P, vp, vp, vp, vp]
+        lib.moba_gate_topk_noalloc.restype = ctypes.c_int
         lib.moba_launches_per_forward.argtypes = [P]
         lib.moba_launches_per_forward.restype = ctypes.c_int
         for f in ("moba_pool_keys", "moba_gate_topk", "moba_attn_fwd", "moba_fwd", "moba_route",
@@ -193,6 +195,11 @@ def moba_attn_self_merge(p: MobaParams, Q, K, V, sel, workspace, O, LSE, stream=
     _check(load().moba_attn_self_merge(p.ref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(sel), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _ptr(O), _ptr(LSE),
                                        _stream(stream)))
+
+
+def moba_gate_topk_noalloc(p: MobaParams, Q, Kbar, sel, stream=None) -> None:
+    """moba_gate_topk for callers without an allocator: scratch is a fixed array in the library."""
+    _check(load().moba_gate_topk_noalloc(p.ref(), _ptr(Q), _ptr(Kbar), _ptr(sel), _stream(stream)))
 
 
 def moba_launches_per_forward(p: MobaParams) -> int:

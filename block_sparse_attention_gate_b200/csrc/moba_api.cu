@@ -366,4 +366,64 @@ moba_status moba_read_device_error(int32_t* value, int clear) {
   return MOBA_OK;
 }
 
+// ---------------------------------------------------------------------------------------
+// Gate without caller scratch.  The tensor-core gate needs scratch for the bf16 hi/lo split of
+// the pooled keys; this variant keeps it in a fixed device array compiled into the library,
+// so the caller passes only inputs and outputs and nothing here allocates.
+}  // extern "C"
+
+namespace {
+constexpr size_t kNoAllocMaxKbarElems = (size_t)1 << 21;  // hi + lo: 2 x 2^21 bf16 = 8 MiB
+}  // namespace
+
+static __device__ __align__(256) __nv_bfloat16 g_gate_scratch[2 * kNoAllocMaxKbarElems];
+
+namespace {
+__nv_bfloat16* g_gate_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_gate_scratch on the current device, looked up once per device (the
+// host-side name of the array is only a stand-in, never a device address).
+moba_status gate_scratch(__nv_bfloat16** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOBA_ERR_DEVICE, "device ordinal %d out of range", dev);
+  if (!g_gate_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_gate_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(gate scratch)");
+    g_gate_scratch_ptr[dev] = static_cast<__nv_bfloat16*>(ptr);
+  }
+  *out = g_gate_scratch_ptr[dev];
+  return MOBA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+moba_status moba_gate_topk_noalloc(const moba_params* p, const void* Q, const float* Kbar, int32_t* sel,
+                                   void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0) return MOBA_OK;
+  const size_t elems = (size_t)g.num_seqs * g.MB * g.Hkv * g.D;
+  if (elems > kNoAllocMaxKbarElems)
+    return fail(MOBA_ERR_UNSUPPORTED,
+                "moba_gate_topk_noalloc: num_seqs * ceil(max_seqlen / block_size) * num_kv_heads * head_dim = "
+                "%zu exceeds the built-in scratch limit of %zu; use moba_gate_topk with a workspace",
+                elems, kNoAllocMaxKbarElems);
+  MOBA_TRY(check_ptr(Q, "Q", true));
+  MOBA_TRY(check_ptr(Kbar, "Kbar", true));
+  MOBA_TRY(check_ptr(sel, "sel", true));
+  MOBA_TRY(check_device(&g));
+  __nv_bfloat16* scratch = nullptr;
+  MOBA_TRY(gate_scratch(&scratch));
+  moba::Work w{};
+  w.kbar_hi = scratch;
+  w.kbar_lo = scratch + kNoAllocMaxKbarElems;
+  cudaError_t e = moba::launch_gate(g, (const __nv_bfloat16*)Q, Kbar, sel, w, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOBA_OK : cuda_fail(e, "gate launch");
+}
+
 }  // extern "C"

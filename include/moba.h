@@ -147,6 +147,29 @@ MOBA_API moba_status moba_attn_self_merge(const moba_params* p, const void* Q, c
                                           const void* V, const int32_t* sel, void* workspace,
                                           size_t workspace_bytes, void* O, float* LSE, void* stream);
 
+/*
+ * moba_gate_topk without a workspace argument.  The MoBA pages have no counterpart: this is
+ * an interface convenience, not part of the method.  Same inputs, outputs and results as
+ * moba_gate_topk, for callers that cannot allocate device memory: code that enqueues work
+ * while a CUDA graph is being captured (cudaMalloc is not allowed then), serving runtimes
+ * that forbid allocation after start-up to keep memory use fixed, and host programs that
+ * receive raw device pointers but no allocator.  The gate's scratch (the bf16 hi/lo split
+ * of Kbar) lives in one device array of MOBA_NOALLOC_MAX_KBAR_ELEMS * 4 bytes (8 MiB) that
+ * is compiled into the library; every GPU that loads the library holds it until exit.
+ *  - Limit: num_seqs * ceil(max_seqlen / block_size) * num_kv_heads * head_dim must not
+ *    exceed MOBA_NOALLOC_MAX_KBAR_ELEMS (2^21; a 1M-token sequence with 8 KV heads of
+ *    dimension 128 at block size 2048 needs 2^19); larger problems get MOBA_ERR_UNSUPPORTED.
+ *  - The first call on each device looks up the array's device address (a CUDA runtime
+ *    query, no allocation); make that first call before any stream capture begins.
+ *  - All calls share the one array and it keeps the last call's contents; every element a
+ *    call reads is written earlier in the same call, so nothing needs clearing.  Calls
+ *    whose kernels overlap on the GPU (other streams, other host threads) race on it and
+ *    must be serialised by the caller.
+ */
+#define MOBA_NOALLOC_MAX_KBAR_ELEMS (1u << 21)
+MOBA_API moba_status moba_gate_topk_noalloc(const moba_params* p, const void* Q, const float* Kbar,
+                                            int32_t* sel, void* stream);
+
 /* Kernel launches one moba_fwd enqueues for these params (host only; -1 if invalid). */
 MOBA_API int moba_launches_per_forward(const moba_params* p);
 
