@@ -28,12 +28,15 @@ namespace moba {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kRows = 128;  // query rows per CTA (M)
-constexpr int kBN = 128;    // keys per chunk (N of S, K of PV)
+constexpr int kThreads = 320;  // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA
+constexpr int kRows = 128;     // query rows per tile (M); two tiles per CTA
+constexpr int kBN = 128;       // keys per chunk (N of S, K of PV)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256;
+constexpr uint32_t kColS = 0;      // S of tile t at kColS + 128 t
+constexpr uint32_t kColP = 0;      // P of tile t (bf16 pairs) aliased at S + 0 .. S + 63
+constexpr uint32_t kColO = 256;    // O of tile t at kColO + 128 t
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleLog2 = 8.f;  // rescale O only when a row max grows by more than 2^8
 
 struct AttnArgs {
   Geom g;
@@ -46,21 +49,34 @@ struct AttnArgs {
   float* part_lse;
   __nv_bfloat16* O;
   float* LSE;
+  int own_head_pairs;  // own mode: tiles are heads (2p, 2p+1) of one group (else query tiles 2p, 2p+1)
 };
 
 template <int D>
 struct Layout {
   static constexpr int kTile = kRows * D * 2;  // bytes of a [128 x D] bf16 tile
-  static constexpr int kQ = 0;
-  static constexpr int kK0 = kQ + kTile;
-  static constexpr int kV0 = kK0 + 2 * kTile;
-  static constexpr int kP = kV0 + 2 * kTile;
-  static constexpr int kBar = kP + kRows * kBN * 2;
+  static constexpr int kQ = 0;                 // two tiles
+  static constexpr int kK0 = kQ + 2 * kTile;   // two stages
+  static constexpr int kV0 = kK0 + 2 * kTile;  // two stages
+  static constexpr int kBar = kV0 + 2 * kTile;
   static constexpr int kBytes = kBar + 256;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
-enum Bar { kQFull = 0, kKVFull0, kKVFull1, kKVEmpty0, kKVEmpty1, kSFull0, kSFull1, kSFree0, kSFree1, kPFull, kPVDone, kDone, kNumBars };
+enum Bar {
+  kQFull = 0, kKFull0, kKFull1, kKEmpty0, kKEmpty1, kVFull0, kVFull1, kVEmpty0, kVEmpty1,
+  kSFull0, kSFull1, kPFull0, kPFull1, kOFull0, kOFull1, kDone, kNumBars
+};
+
+// One tile's row source and causal geometry.
+struct TileInfo {
+  int64_t qrow_base;  // own mode: Q row of token q0 (t * Hq + h) ...
+  int32_t q0;         // own mode: first token
+  int h;              // own mode: query head
+  int nrows;          // valid rows (0..128)
+  int diag;           // own mode: index of the diagonal chunk
+  int32_t row_start;  // past mode: first routed position
+};
 
 template <int D, bool kOwn>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -74,9 +90,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ------------------------------------------------------------- work item
-  int gk, h = 0, s;
-  int32_t key0, nrows, row_start = 0, q0 = 0, i_blk = 0;
-  int nchunks;
+  int gk, s, i_blk = 0, nchunks;
+  int32_t key0;
+  TileInfo ti[2];
   if constexpr (!kOwn) {
     const int32_t total = __ldg(a.tile_off + g.nbk);
     const int32_t tile = (int32_t)blockIdx.x;
@@ -89,146 +105,189 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t b = (int32_t)(lo % g.MB);
     s = (int)((lo / g.MB) % g.num_seqs);
     gk = (int)(lo / ((int64_t)g.MB * g.num_seqs));
-    row_start = __ldg(a.offsets + lo) + (tile - __ldg(a.tile_off + lo)) * kRows;
-    nrows = min(kRows, __ldg(a.offsets + lo + 1) - row_start);
+    const int32_t rs = __ldg(a.offsets + lo) + (tile - __ldg(a.tile_off + lo)) * (2 * kRows);
+    const int32_t re = __ldg(a.offsets + lo + 1);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      ti[t].row_start = rs + t * kRows;
+      ti[t].nrows = max(0, min(kRows, re - ti[t].row_start));
+      ti[t].diag = 1 << 30;
+      ti[t].qrow_base = 0; ti[t].q0 = 0; ti[t].h = 0;
+    }
     key0 = seq_start(g, s) + b * g.bs;
     nchunks = g.bs / kBN;
   } else {
     const int per_blk = g.bs / kRows;
-    i_blk = blockIdx.x / per_blk;
-    const int qt = blockIdx.x - i_blk * per_blk;
     s = blockIdx.y;
-    h = blockIdx.z;
-    gk = h / g.G;
     const int32_t ts = seq_start(g, s), te = seq_end(g, s);
+    if (a.own_head_pairs) {
+      i_blk = blockIdx.x / per_blk;
+      const int qt = blockIdx.x - i_blk * per_blk;
+      const int32_t q0 = ts + i_blk * g.bs + qt * kRows;
+      if (q0 >= te) return;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        ti[t].h = 2 * blockIdx.z + t;
+        ti[t].q0 = q0;
+        ti[t].nrows = min(kRows, te - q0);
+        ti[t].diag = qt;
+        ti[t].row_start = 0;
+      }
+      nchunks = qt + 1;
+    } else {
+      const int pairs = (per_blk + 1) / 2;
+      i_blk = blockIdx.x / pairs;
+      const int qp = blockIdx.x - i_blk * pairs;
+      const int32_t q0 = ts + i_blk * g.bs + 2 * qp * kRows;
+      if (q0 >= te) return;
+      const int qt1 = 2 * qp + 1;
+      const bool has1 = qt1 < per_blk && q0 + kRows < te;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        ti[t].h = blockIdx.z;
+        ti[t].q0 = q0 + t * kRows;
+        ti[t].nrows = (t == 0 || has1) ? max(0, min(kRows, te - ti[t].q0)) : 0;
+        ti[t].diag = 2 * qp + t;
+        ti[t].row_start = 0;
+      }
+      nchunks = has1 ? qt1 + 1 : 2 * qp + 1;
+    }
+    gk = ti[0].h / g.G;
     key0 = ts + i_blk * g.bs;
-    q0 = key0 + qt * kRows;
-    if (q0 >= te) return;
-    nrows = min(kRows, te - q0);
-    nchunks = qt + 1;
   }
 
   // ------------------------------------------------------------- setup
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
     tc_fence_before();
   }
   if (tid == 0) {
-    mbar_init(&bars[kQFull], kRows);
-    mbar_init(&bars[kKVFull0], 1);
-    mbar_init(&bars[kKVFull1], 1);
-    mbar_init(&bars[kKVEmpty0], 1);
-    mbar_init(&bars[kKVEmpty1], 1);
-    mbar_init(&bars[kSFull0], 1);
-    mbar_init(&bars[kSFull1], 1);
-    mbar_init(&bars[kSFree0], kRows);
-    mbar_init(&bars[kSFree1], kRows);
-    mbar_init(&bars[kPFull], kRows);
-    mbar_init(&bars[kPVDone], 1);
+    mbar_init(&bars[kQFull], 2 * kRows);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&bars[kKFull0 + q], 1);
+      mbar_init(&bars[kKEmpty0 + q], 1);
+      mbar_init(&bars[kVFull0 + q], 1);
+      mbar_init(&bars[kVEmpty0 + q], 1);
+      mbar_init(&bars[kSFull0 + q], 1);
+      mbar_init(&bars[kPFull0 + q], kRows);
+      mbar_init(&bars[kOFull0 + q], 1);
+    }
     mbar_init(&bars[kDone], 1);
     fence_mbar_init();
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t sQ = smem_u32(smem + L::kQ);
-  const uint32_t sK0 = smem_u32(smem + L::kK0);
-  const uint32_t sV0 = smem_u32(smem + L::kV0);
-  const uint32_t sP = smem_u32(smem + L::kP);
   bool ok = true;
 
-  if (warp < 4) {
-    // ========================================================= softmax warps
-    const int r = tid;
+  if (warp < 8) {
+    // ========================================================= softmax warpgroups
+    const int t = warp >> 2;           // tile
+    const int r = tid & (kRows - 1);   // row = TMEM lane
+    const TileInfo& T_ = ti[t];
     int64_t qrow = -1;
     int32_t e = -1;
-    if (r < nrows) {
+    if (r < T_.nrows) {
       if constexpr (!kOwn) {
-        e = __ldg(a.rows + row_start + r);
+        e = __ldg(a.rows + T_.row_start + r);
         qrow = e / (g.k - 1);
       } else {
-        qrow = (int64_t)(q0 + r) * g.Hq + h;
+        qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
       }
     }
-    {  // gather this row of Q into the swizzled tile (zeros for padding rows)
+    {  // gather this row of Q into tile t (zeros for padding rows)
       const __nv_bfloat16* src = qrow >= 0 ? a.Q + qrow * D : a.Q;
       const uint32_t nb = qrow >= 0 ? 16u : 0u;
+      const uint32_t sQ = smem_u32(smem + L::kQ + t * L::kTile);
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) cp_async_16(sQ + sw128_offset(r, c, kRows), src + c * 8, nb);
       cp_async_wait_all();
       fence_proxy_async_smem();
       mbar_arrive(&bars[kQFull]);
     }
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + kColS + t * kBN;
+    const uint32_t tP = tS + kColP;
+    const uint32_t tO = tmem + lane_off + kColO + t * 128;
     const float c2 = g.scale_log2;
     float m = -INFINITY, l = 0.f;
     for (int j = 0; j < nchunks && ok; ++j) {
-      const int sb = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull0 + sb], (j >> 1) & 1, g.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull0 + t], j & 1, g.err));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + kColS0 + sb * kBN + c * 32, sr[c]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars[kSFree0 + sb]);
-      const bool diag = kOwn && (j == nchunks - 1);
+      // pass 1: row max of the scaled logits (log2 units), causal mask in the own block
+      const int lim = kOwn ? (j < T_.diag ? kBN : (j == T_.diag ? r + 1 : 0)) : kBN;
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t sa[32], sb[32];
+        tmem_ld32(tS + cc * 64, sa);
+        tmem_ld32(tS + cc * 64 + 32, sb);
+        tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          float v = __uint_as_float(sr[c][x]) * c2;
-          if (diag && (c * 32 + x) > r) v = -INFINITY;
-          sr[c][x] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          const bool ka = !kOwn || (cc * 64 + x) < lim, kb = !kOwn || (cc * 64 + 32 + x) < lim;
+          mx = fmaxf(mx, ka ? __uint_as_float(sa[x]) : -INFINITY);
+          mx = fmaxf(mx, kb ? __uint_as_float(sb[x]) : -INFINITY);
         }
-      const float m_new = fmaxf(m, mx);
-      const float alpha = ex2(m - m_new);
-      float rs = 0.f;
-      uint32_t pk[64];
+      }
+      mx *= c2;
+      // running max: rescale the TMEM accumulator only when it grows by more than 2^8
+      // (p <= 256 otherwise, harmless in fp32 sums and bf16 P).  At this point the previous
+      // PV of this tile has completed: the MMA that produced this S was issued after it.
+      if (j == 0) {
+        m = mx;
+      } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
+        const float m_new = fmaxf(m, mx);
+        const float alpha = ex2(m - m_new);
+        l *= alpha;
+        m = m_new;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+          tmem_st32(tO + c * 32, o);
+        }
+      }
+      // pass 2: p = 2^(s*c2 - m); P (bf16 pairs) overwrites S columns already consumed
+      float rs = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t sa[32], sb[32], pk[32];
+        tmem_ld32(tS + cc * 64, sa);
+        tmem_ld32(tS + cc * 64 + 32, sb);
+        tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
-          const float p0 = ex2(__uint_as_float(sr[c][x]) - m_new);
-          const float p1 = ex2(__uint_as_float(sr[c][x + 1]) - m_new);
+          float p0 = ex2(fmaf(__uint_as_float(sa[x]), c2, -m));
+          float p1 = ex2(fmaf(__uint_as_float(sa[x + 1]), c2, -m));
+          if (kOwn && (cc * 64 + x) >= lim) p0 = 0.f;
+          if (kOwn && (cc * 64 + x + 1) >= lim) p1 = 0.f;
           rs += p0 + p1;
-          pk[(c * 32 + x) >> 1] = pack_bf16x2(p0, p1);
+          pk[x >> 1] = pack_bf16x2(p0, p1);
         }
-      l = l * alpha + rs;
-      m = m_new;
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kPVDone], (j - 1) & 1, g.err));
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_off + kColO + c * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(tmem + lane_off + kColO + c * 32, o);
-          }
-          tmem_wait_st();
+        for (int x = 0; x < 32; x += 2) {
+          float p0 = ex2(fmaf(__uint_as_float(sb[x]), c2, -m));
+          float p1 = ex2(fmaf(__uint_as_float(sb[x + 1]), c2, -m));
+          if (kOwn && (cc * 64 + 32 + x) >= lim) p0 = 0.f;
+          if (kOwn && (cc * 64 + 32 + x + 1) >= lim) p1 = 0.f;
+          rs += p0 + p1;
+          pk[16 + (x >> 1)] = pack_bf16x2(p0, p1);
         }
+        tmem_st32(tP + cc * 32, pk);
       }
-      uint8_t* pbase = smem + L::kP;
-#pragma unroll
-      for (int c16 = 0; c16 < kBN / 8; ++c16) {
-        uint4 v = make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
-        *reinterpret_cast<uint4*>(pbase + sw128_offset(r, c16, kRows)) = v;
-      }
-      fence_proxy_async_smem();
+      l += rs;
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[kPFull]);
+      mbar_arrive(&bars[kPFull0 + t]);
     }
     // ------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kPVDone], (nchunks - 1) & 1, g.err));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull0 + t], 0, g.err));
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.f / l;
@@ -237,9 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_off + kColO + c * 32, o);
+          tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
-          if (r < nrows) {
+          if (r < T_.nrows) {
             float4* dst = reinterpret_cast<float4*>(a.part_o + (int64_t)e * D + c * 32);
 #pragma unroll
             for (int x = 0; x < 32; x += 4)
@@ -247,14 +306,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         __uint_as_float(o[x + 2]) * inv_l, __uint_as_float(o[x + 3]) * inv_l);
           }
         }
-        if (r < nrows) a.part_lse[e] = lse_row;
+        if (r < T_.nrows) a.part_lse[e] = lse_row;
       } else {
         // online-softmax merge of the own-block result with the row's past partials
         float M = lse_row;
         int32_t pe[kMaxTopK];
         float pl[kMaxTopK];
         int np = 0;
-        if (r < nrows) {
+        if (r < T_.nrows) {
           for (int slot = 1; slot < g.k; ++slot) {
             const int32_t b = __ldg(a.sel + qrow * g.k + slot);
             if (b >= 0 && b < i_blk) {
@@ -276,9 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_off + kColO + c * 32, o);
+          tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
-          if (r < nrows) {
+          if (r < T_.nrows) {
             float acc[32];
 #pragma unroll
             for (int x = 0; x < 32; ++x) acc[x] = __uint_as_float(o[x]) * a_self;
@@ -301,28 +360,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        pack_bf16x2(acc[x + 4], acc[x + 5]), pack_bf16x2(acc[x + 6], acc[x + 7]));
           }
         }
-        if (r < nrows) a.LSE[qrow] = M + __logf(sumw);
+        if (r < T_.nrows) a.LSE[qrow] = M + __logf(sumw);
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     // ========================================================= TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       for (int j = 0; j < nchunks && ok; ++j) {
         const int st = j & 1, u = j >> 1;
-        if (u > 0) {
-          ok = mbar_wait(&bars[kKVEmpty0 + st], (u - 1) & 1, g.err);
-          if (!ok) break;
-        }
-        uint64_t* full = &bars[kKVFull0 + st];
-        mbar_expect_tx(full, 2u * L::kTile);
-        const int t = key0 + j * kBN;
+        const int tok = key0 + j * kBN;
+        if (u > 0) ok = mbar_wait(&bars[kKEmpty0 + st], (u - 1) & 1, g.err);
+        if (!ok) break;
+        mbar_expect_tx(&bars[kKFull0 + st], L::kTile);
 #pragma unroll
-        for (int hh = 0; hh < D / 64; ++hh) {
-          tma_load_3d(smem + L::kK0 + st * L::kTile + hh * kRows * 128, &tmK, full, hh * 64, gk, t);
-          tma_load_3d(smem + L::kV0 + st * L::kTile + hh * kRows * 128, &tmV, full, hh * 64, gk, t);
-        }
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_3d(smem + L::kK0 + st * L::kTile + hh * kRows * 128, &tmK, &bars[kKFull0 + st], hh * 64, gk, tok);
+        if (u > 0) ok = mbar_wait(&bars[kVEmpty0 + st], (u - 1) & 1, g.err);
+        if (!ok) break;
+        mbar_expect_tx(&bars[kVFull0 + st], L::kTile);
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_3d(smem + L::kV0 + st * L::kTile + hh * kRows * 128, &tmV, &bars[kVFull0 + st], hh * 64, gk, tok);
       }
     }
   } else {
@@ -330,39 +390,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kRows, kBN, false, false);
       constexpr uint32_t idO = idesc_bf16(kRows, D, false, true);
-      auto issue_pv = [&](int c) -> bool {
-        if (!mbar_wait(&bars[kPFull], c & 1, g.err)) return false;
-        tc_fence_after();
-        const uint32_t vb = sV0 + (c & 1) * L::kTile;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(sP + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(vb + kk * 2048, kRows * 128, 1024);
-          mma_bf16_ss(tmem + kColO, ad, bd, idO, (c > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&bars[kPVDone]);
-        mma_commit(&bars[kKVEmpty0 + (c & 1)]);
-        return true;
-      };
-      ok = mbar_wait(&bars[kQFull], 0, g.err);
-      for (int j = 0; j < nchunks && ok; ++j) {
-        const int st = j & 1, sb = j & 1;
-        ok = mbar_wait(&bars[kKVFull0 + st], (j >> 1) & 1, g.err);
-        if (ok && j >= 2) ok = mbar_wait(&bars[kSFree0 + sb], ((j >> 1) - 1) & 1, g.err);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kb = sK0 + st * L::kTile;
+      const uint32_t sQ = smem_u32(smem + L::kQ);
+      const uint32_t sK0 = smem_u32(smem + L::kK0);
+      const uint32_t sV0 = smem_u32(smem + L::kV0);
+      auto issue_s = [&](int t, int j) {
+        const uint32_t qb = sQ + t * L::kTile, kb = sK0 + (j & 1) * L::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(kb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
-          mma_bf16_ss(tmem + kColS0 + sb * kBN, ad, bd, idS, kk > 0 ? 1u : 0u);
+          const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+          mma_bf16_ss(tmem + kColS + t * kBN, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idS,
+                      kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars[kSFull0 + sb]);
-        if (j >= 1) ok = issue_pv(j - 1);
+        mma_commit(&bars[kSFull0 + t]);
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t vb = sV0 + (j & 1) * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_bf16_ts(tmem + kColO + t * 128, tmem + kColS + t * kBN + kColP + kk * 8,
+                      sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      ok = mbar_wait(&bars[kQFull], 0, g.err) && mbar_wait(&bars[kKFull0], 0, g.err);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        mma_commit(&bars[kKEmpty0]);
       }
-      if (ok) ok = issue_pv(nchunks - 1);
-      // every MMA issued above has completed once kDone fires
+      for (int j = 0; j < nchunks && ok; ++j) {
+        const bool more = j + 1 < nchunks;
+        ok = mbar_wait(&bars[kVFull0 + (j & 1)], (j >> 1) & 1, g.err) && mbar_wait(&bars[kPFull0], j & 1, g.err);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (!more) mma_commit(&bars[kOFull0]);
+        if (more) {
+          ok = mbar_wait(&bars[kKFull0 + ((j + 1) & 1)], ((j + 1) >> 1) & 1, g.err);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        ok = mbar_wait(&bars[kPFull1], j & 1, g.err);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        mma_commit(&bars[kVEmpty0 + (j & 1)]);
+        if (!more) mma_commit(&bars[kOFull1]);
+        if (more) {
+          issue_s(1, j + 1);
+          mma_commit(&bars[kKEmpty0 + ((j + 1) & 1)]);
+        }
+      }
       mma_commit(&bars[kDone]);
       mbar_wait(&bars[kDone], 0, g.err);
     }
@@ -370,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ------------------------------------------------------------- teardown
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -378,13 +456,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool kOwn>
 cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
-                      const int32_t* sel, const Work& w, __nv_bfloat16* O, float* LSE, dim3 grid, cudaStream_t st) {
+                      const int32_t* sel, const Work& w, __nv_bfloat16* O, float* LSE, dim3 grid, int head_pairs,
+                      cudaStream_t st) {
   CUtensorMap tk, tv;
   cudaError_t e = make_rows_map(&tk, K, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
   e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
-  AttnArgs a{g, Q, sel, w.offsets, w.tile_off, w.rows, w.part_o, w.part_lse, O, LSE};
+  AttnArgs a{g, Q, sel, w.offsets, w.tile_off, w.rows, w.part_o, w.part_lse, O, LSE, head_pairs};
   const int smem = Layout<D>::kAlloc;
   e = cudaFuncSetAttribute(attn_tc_kernel<D, kOwn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -397,19 +476,22 @@ cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16
 cudaError_t launch_attn_past(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                              const __nv_bfloat16* V, const Work& w, cudaStream_t st) {
   if (g.T == 0 || g.k < 2 || g.R == 0) return cudaSuccess;
-  const int64_t tiles = (g.R + kRows - 1) / kRows + g.nbk;  // upper bound of the routed tile count
+  const int64_t tiles = (g.R + kPastTileRows - 1) / kPastTileRows + g.nbk;  // bound on routed tile pairs
   dim3 grid((unsigned)tiles);
-  if (g.D == 64) return launch_tc<64, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, grid, st);
-  return launch_tc<128, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, grid, st);
+  if (g.D == 64) return launch_tc<64, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, grid, 0, st);
+  return launch_tc<128, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, grid, 0, st);
 }
 
 cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                              const __nv_bfloat16* V, const int32_t* sel, const Work& w,
                              __nv_bfloat16* O, float* LSE, cudaStream_t st) {
   if (g.T == 0) return cudaSuccess;
-  dim3 grid((unsigned)(g.MB * (g.bs / kRows)), (unsigned)g.num_seqs, (unsigned)g.Hq);
-  if (g.D == 64) return launch_tc<64, true>(g, Q, K, V, sel, w, O, LSE, grid, st);
-  return launch_tc<128, true>(g, Q, K, V, sel, w, O, LSE, grid, st);
+  const int per_blk = g.bs / kRows;
+  const int head_pairs = (g.G % 2 == 0) ? 1 : 0;
+  dim3 grid = head_pairs ? dim3((unsigned)(g.MB * per_blk), (unsigned)g.num_seqs, (unsigned)(g.Hq / 2))
+                         : dim3((unsigned)(g.MB * ((per_blk + 1) / 2)), (unsigned)g.num_seqs, (unsigned)g.Hq);
+  if (g.D == 64) return launch_tc<64, true>(g, Q, K, V, sel, w, O, LSE, grid, head_pairs, st);
+  return launch_tc<128, true>(g, Q, K, V, sel, w, O, LSE, grid, head_pairs, st);
 }
 
 int launches_per_forward(const Geom& g) {

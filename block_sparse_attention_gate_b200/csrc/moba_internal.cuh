@@ -9,6 +9,8 @@
 namespace moba {
 
 constexpr int kMaxTopK = 16;
+// Routed rows per past-block attention CTA (two 128-row tiles); route.cu tiles buckets by it.
+constexpr int kPastTileRows = 256;
 
 // Problem geometry as the kernels see it (passed by value).
 struct Geom {

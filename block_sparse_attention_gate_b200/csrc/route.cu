@@ -129,7 +129,7 @@ cudaError_t launch_route_tiles(const Geom& g, const int32_t* sel, const Work& w,
 }
 
 cudaError_t launch_route(const Geom& g, const int32_t* sel, const Work& w, cudaStream_t st) {
-  return launch_route_tiles(g, sel, w, 128, st);
+  return launch_route_tiles(g, sel, w, kPastTileRows, st);
 }
 
 }  // namespace moba
