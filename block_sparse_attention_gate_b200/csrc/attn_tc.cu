@@ -28,7 +28,15 @@ namespace moba {
 
 namespace {
 
-constexpr int kThreads = 320;  // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA
+constexpr int kThreads = 384;  // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA, 10-11 idle
+// Register split (setmaxnreg): the kernel is compiled for kLaunchRegs per thread; the third
+// warpgroup gives registers back so the two softmax warpgroups can hold a full S row.
+// 2 * 128 * kSoftmaxRegs + 128 * kOtherRegs must not exceed 384 * kLaunchRegs (checked on
+// the host against the compiled register count before every launch).
+constexpr uint32_t kLaunchRegs = 168;
+constexpr uint32_t kSoftmaxRegs = 216;
+constexpr uint32_t kOtherRegs = 72;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= 384 * kLaunchRegs, "register split too large");
 constexpr int kRows = 128;     // query rows per tile (M); two tiles per CTA
 constexpr int kBN = 128;       // keys per chunk (N of S, K of PV)
 constexpr uint32_t kTmemCols = 512;
@@ -180,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
+  if (warp >= 8) regs_dec<kOtherRegs>(); else regs_inc<kSoftmaxRegs>();
 
   if (warp < 8) {
     // ========================================================= softmax warpgroups
@@ -216,21 +225,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull0 + t], j & 1, g.err));
       if (!ok) break;
       tc_fence_after();
-      // pass 1: row max of the scaled logits (log2 units), causal mask in the own block
-      const int lim = kOwn ? (j < T_.diag ? kBN : (j == T_.diag ? r + 1 : 0)) : kBN;
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+      tmem_wait_ld();
+      // scaled-logit row max (log2 units); the causal mask applies to the diagonal chunk only
+      // (keys after the diagonal chunk, in the query-tile-pair layout, are all masked)
+      const bool masked = kOwn && j >= T_.diag;
+      const int lim = (kOwn && j == T_.diag) ? r + 1 : (masked ? 0 : kBN);
       float mx = -INFINITY;
+      if (!masked) {
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sa[32], sb[32];
-        tmem_ld32(tS + cc * 64, sa);
-        tmem_ld32(tS + cc * 64 + 32, sb);
-        tmem_wait_ld();
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const bool ka = !kOwn || (cc * 64 + x) < lim, kb = !kOwn || (cc * 64 + 32 + x) < lim;
-          mx = fmaxf(mx, ka ? __uint_as_float(sa[x]) : -INFINITY);
-          mx = fmaxf(mx, kb ? __uint_as_float(sb[x]) : -INFINITY);
-        }
+          for (int x = 0; x < 32; ++x) mx = fmaxf(mx, __uint_as_float(sr[c][x]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            if (c * 32 + x < lim) mx = fmaxf(mx, __uint_as_float(sr[c][x]));
       }
       mx *= c2;
       // running max: rescale the TMEM accumulator only when it grows by more than 2^8
@@ -253,31 +267,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(tO + c * 32, o);
         }
       }
-      // pass 2: p = 2^(s*c2 - m); P (bf16 pairs) overwrites S columns already consumed
+      // p = 2^(s*c2 - m); P (bf16 pairs) overwrites the first 64 S columns (S is in registers)
       float rs = 0.f;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sa[32], sb[32], pk[32];
-        tmem_ld32(tS + cc * 64, sa);
-        tmem_ld32(tS + cc * 64 + 32, sb);
-        tmem_wait_ld();
+        uint32_t pk[32];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(sa[x]), c2, -m));
-          float p1 = ex2(fmaf(__uint_as_float(sa[x + 1]), c2, -m));
-          if (kOwn && (cc * 64 + x) >= lim) p0 = 0.f;
-          if (kOwn && (cc * 64 + x + 1) >= lim) p1 = 0.f;
-          rs += p0 + p1;
-          pk[x >> 1] = pack_bf16x2(p0, p1);
-        }
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int c = 2 * cc + h2;
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(sb[x]), c2, -m));
-          float p1 = ex2(fmaf(__uint_as_float(sb[x + 1]), c2, -m));
-          if (kOwn && (cc * 64 + 32 + x) >= lim) p0 = 0.f;
-          if (kOwn && (cc * 64 + 32 + x + 1) >= lim) p1 = 0.f;
-          rs += p0 + p1;
-          pk[16 + (x >> 1)] = pack_bf16x2(p0, p1);
+          for (int x = 0; x < 32; x += 2) {
+            float p0 = ex2(fmaf(__uint_as_float(sr[c][x]), c2, -m));
+            float p1 = ex2(fmaf(__uint_as_float(sr[c][x + 1]), c2, -m));
+            if (masked) {
+              if (c * 32 + x >= lim) p0 = 0.f;
+              if (c * 32 + x + 1 >= lim) p1 = 0.f;
+            }
+            rs += p0 + p1;
+            pk[16 * h2 + (x >> 1)] = pack_bf16x2(p0, p1);
+          }
         }
         tmem_st32(tP + cc * 32, pk);
       }
@@ -467,6 +475,11 @@ cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16
   const int smem = Layout<D>::kAlloc;
   e = cudaFuncSetAttribute(attn_tc_kernel<D, kOwn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  // the setmaxnreg split must fit in what the launch reserves, or the increase never returns
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D, kOwn>);
+  if (e != cudaSuccess) return e;
+  if ((uint32_t)fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
   attn_tc_kernel<D, kOwn><<<grid, kThreads, smem, st>>>(tk, tv, a);
   return cudaGetLastError();
 }
