@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(smem + L::kV0 + st * L::kTile + hh * kRows * 128, &tmV, &bars[kVFull0 + st], hh * 64, gk, tok);
       }
     }
-  } else {
+  } else if (warp == 9) {
     // ========================================================= MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kRows, kBN, false, false);
