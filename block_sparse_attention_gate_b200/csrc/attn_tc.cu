@@ -277,10 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c = 2 * cc + h2;
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
-            // one exponential in four on the FMA pipe, the rest on MUFU
             float p0 = ex2(fmaf(__uint_as_float(sr[c][x]), c2, -m));
-            float p1 = (x & 2) ? ex2_poly(fmaf(__uint_as_float(sr[c][x + 1]), c2, -m))
-                               : ex2(fmaf(__uint_as_float(sr[c][x + 1]), c2, -m));
+            float p1 = ex2(fmaf(__uint_as_float(sr[c][x + 1]), c2, -m));
             if (masked) {
               if (c * 32 + x >= lim) p0 = 0.f;
               if (c * 32 + x + 1 >= lim) p1 = 0.f;

@@ -201,25 +201,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// 2^x on the FMA pipe (for x <= 127), to take part of the softmax exponentials off the MUFU
-// unit.  Exact range reduction x = n + f with n = rint(x), |f| <= 1/2 (adding 1.5 * 2^23
-// leaves rint(x) in the low mantissa bits), then 2^f from a degree-3 polynomial whose
-// coefficients come from our own relative-error (Lawson / reweighted least-squares) fit on
-// [-1/2, 1/2]: max relative error 7.5e-5, far below the bf16 rounding of P (2^-9).  2^n is
-// applied by adding n to the exponent bits; x is clamped at -126 (the result is then
-// below 2^-125, where only its negligible size matters).
-constexpr float kEx2P0 = 0.99992812f, kEx2P1 = 0.69326097f, kEx2P2 = 0.24261054f, kEx2P3 = 0.05517132f;
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float n = t - 12582912.f;
-  const float f = x - n;
-  float p = fmaf(kEx2P3, f, kEx2P2);
-  p = fmaf(p, f, kEx2P1);
-  p = fmaf(p, f, kEx2P0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
