@@ -233,19 +233,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (keys after the diagonal chunk, in the query-tile-pair layout, are all masked)
       const bool masked = kOwn && j >= T_.diag;
       const int lim = (kOwn && j == T_.diag) ? r + 1 : (masked ? 0 : kBN);
-      float mx = -INFINITY;
+      // eight independent running maxima keep the dependency chain short
+      float mv[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mv[q] = -INFINITY;
       if (!masked) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int x = 0; x < 32; ++x) mx = fmaxf(mx, __uint_as_float(sr[c][x]));
+          for (int x = 0; x < 32; ++x) mv[x & 7] = fmaxf(mv[x & 7], __uint_as_float(sr[c][x]));
       } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int x = 0; x < 32; ++x)
-            if (c * 32 + x < lim) mx = fmaxf(mx, __uint_as_float(sr[c][x]));
+            if (c * 32 + x < lim) mv[x & 7] = fmaxf(mv[x & 7], __uint_as_float(sr[c][x]));
       }
+      float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])), fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
       mx *= c2;
       // running max: rescale the TMEM accumulator only when it grows by more than 2^8
       // (p <= 256 otherwise, harmless in fp32 sums and bf16 P).  At this point the previous
@@ -268,7 +272,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // p = 2^(s*c2 - m); P (bf16 pairs) overwrites the first 64 S columns (S is in registers)
-      float rs = 0.f;
+      float rv[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) rv[q] = 0.f;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t pk[32];
@@ -283,12 +289,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (c * 32 + x >= lim) p0 = 0.f;
               if (c * 32 + x + 1 >= lim) p1 = 0.f;
             }
-            rs += p0 + p1;
+            rv[x & 7] += p0;
+            rv[(x & 7) + 1] += p1;
             pk[16 * h2 + (x >> 1)] = pack_bf16x2(p0, p1);
           }
         }
         tmem_st32(tP + cc * 32, pk);
       }
+      const float rs = ((rv[0] + rv[1]) + (rv[2] + rv[3])) + ((rv[4] + rv[5]) + (rv[6] + rv[7]));
       l += rs;
       tmem_wait_st();
       tc_fence_before();
