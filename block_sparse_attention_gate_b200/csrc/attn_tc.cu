@@ -1,33 +1,23 @@
 // MoBA block attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
 //
 // Two modes share one kernel body:
-//   past : work item = two 128-row tiles of routed query rows of one bucket (KV head g,
-//          sequence s, past block b) against the whole block (bs keys: a past block is
-//          complete and fully visible); writes normalised fp32 partials + LSE.
-//   own  : work item = two 128-row query tiles inside one block (two heads of a GQA group,
-//          or two consecutive tiles of one head) against the block's keys up to the
-//          diagonal (causal mask on the diagonal chunk); then each row's past partials are
-//          merged by online softmax and O (bf16) and LSE are written.
+//   past : a CTA takes a tile of up to 128 routed query rows of one bucket (KV head g,
+//          sequence s, past block b), attends the whole block (bs keys; a past block is
+//          complete and fully visible) and writes normalised fp32 partials + LSE.
+//   own  : a CTA takes 128 consecutive tokens of one query head inside one block, attends
+//          the block's keys up to the diagonal (causal mask on the diagonal chunk), then
+//          merges the past partials of every row by online softmax and writes O (bf16) and
+//          LSE.
 // (youleyou.com, "Kimi发布MoBA突破性实现无限上下文", section "PyTorch实现关键要点": attention
 // runs on the own block and on the selected blocks separately and the results are merged by
 // online softmax; zhuoshang.net, "MoBA是什么？…", section "MoBA的技术原理": causal mask inside
 // the current block.)
 //
-// Persistent: one CTA per SM walks the work items (static round-robin); every barrier phase
-// carries over from item to item, K/V loads run ahead across item boundaries, the next item's
-// Q rows are gathered during the current item's last chunk, and an item's epilogue overlaps
-// the next item's first QK^T MMAs.
-//
-// Per 128-key chunk j and tile t:  S_t = Q_t K_j^T     (SS MMA into TMEM)
-//                                  softmax: one thread per row (TMEM lane), P_t as bf16
-//                                  pairs written back over S_t in TMEM
-//                                  O_t += P_t V_j       (TS MMA, P from TMEM)
-// MMA issue order per chunk: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so the tensor core works on
-// one tile while the other tile's softmax runs.  MMAs issued by one thread execute in order,
-// which orders each PV's read of P before the next S overwrites it, and the commit of S_t(j+1)
-// also covers PV_t(j), so a softmax that sees S_t(j+1) may rescale O_t.
-// Warp roles: warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA producer, 9 TMEM owner and
-// MMA issuer, 10-11 idle (they give their registers to the softmax warpgroups).
+// Per 128-key chunk j:  S_j = Q K_j^T  (tcgen05, fp32 in TMEM, double-buffered)
+//                       softmax rows in registers (one thread per row), P_j -> smem (bf16)
+//                       O += P_j V_j    (tcgen05, fp32 accumulator in TMEM)
+// Warp roles: warps 0-3 softmax + epilogue (thread r owns row r = TMEM lane r), warp 4 TMA
+// producer (K/V chunks, two stages), warp 5 TMEM owner + MMA issuer.
 #include <cudaTypedefs.h>
 #include <float.h>
 
@@ -38,7 +28,7 @@ namespace moba {
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 384;  // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA, 10-11 idle
 // Register split (setmaxnreg): the kernel is compiled for kLaunchRegs per thread; the third
 // warpgroup gives registers back so the two softmax warpgroups can hold a full S row.
 // 2 * 128 * kSoftmaxRegs + 128 * kOtherRegs must not exceed 384 * kLaunchRegs (checked on
@@ -47,8 +37,7 @@ constexpr uint32_t kLaunchRegs = 168;
 constexpr uint32_t kSoftmaxRegs = 216;
 constexpr uint32_t kOtherRegs = 72;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= 384 * kLaunchRegs, "register split too large");
-
-constexpr int kRows = 128;     // query rows per tile (M); two tiles per item
+constexpr int kRows = 128;     // query rows per tile (M); two tiles per CTA
 constexpr int kBN = 128;       // keys per chunk (N of S, K of PV)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // S of tile t at kColS + 128 t
@@ -69,7 +58,6 @@ struct AttnArgs {
   __nv_bfloat16* O;
   float* LSE;
   int own_head_pairs;  // own mode: tiles are heads (2p, 2p+1) of one group (else query tiles 2p, 2p+1)
-  int64_t own_items;   // own mode: number of work items
 };
 
 template <int D>
@@ -84,146 +72,19 @@ struct Layout {
 };
 
 enum Bar {
-  kQFull0 = 0, kQFull1, kKFull0, kKFull1, kKEmpty0, kKEmpty1, kVFull0, kVFull1, kVEmpty0, kVEmpty1,
+  kQFull = 0, kKFull0, kKFull1, kKEmpty0, kKEmpty1, kVFull0, kVFull1, kVEmpty0, kVEmpty1,
   kSFull0, kSFull1, kPFull0, kPFull1, kOFull0, kOFull1, kDone, kNumBars
 };
 
-// One work item: two 128-row query tiles against keys [key0, key0 + 128 * nchunks) of KV
-// head gk.
-struct Item {
-  bool valid;
-  int gk, s, i_blk, nchunks;
-  int32_t key0;
-  int32_t row_start[2];  // past: first routed position of each tile
-  int nrows[2];          // valid rows per tile (0..128)
-  int diag[2];           // own: index of each tile's diagonal chunk
-  int32_t q0[2];         // own: first token of each tile
-  int h[2];              // own: query head of each tile
+// One tile's row source and causal geometry.
+struct TileInfo {
+  int64_t qrow_base;  // own mode: Q row of token q0 (t * Hq + h) ...
+  int32_t q0;         // own mode: first token
+  int h;              // own mode: query head
+  int nrows;          // valid rows (0..128)
+  int diag;           // own mode: index of the diagonal chunk
+  int32_t row_start;  // past mode: first routed position
 };
-
-template <bool kOwn>
-__device__ __forceinline__ int64_t num_items(const AttnArgs& a) {
-  if constexpr (!kOwn) return __ldg(a.tile_off + a.g.nbk);
-  else return a.own_items;
-}
-
-// Own-mode items are enumerated longest first (chunk count descending), so the static
-// round-robin over the persistent CTAs finishes with short items.
-template <bool kOwn>
-__device__ __forceinline__ Item decode_item(const AttnArgs& a, int64_t item) {
-  const Geom& g = a.g;
-  Item it;
-  it.valid = true;
-  it.i_blk = 0;
-  if constexpr (!kOwn) {
-    const int32_t tile = (int32_t)item;
-    int64_t lo = 0, hi = g.nbk - 1;  // last bucket whose first tile is <= tile
-    while (lo < hi) {
-      const int64_t mid = (lo + hi + 1) >> 1;
-      if (__ldg(a.tile_off + mid) <= tile) lo = mid; else hi = mid - 1;
-    }
-    const int32_t b = (int32_t)(lo % g.MB);
-    it.s = (int)((lo / g.MB) % g.num_seqs);
-    it.gk = (int)(lo / ((int64_t)g.MB * g.num_seqs));
-    const int32_t rs = __ldg(a.offsets + lo) + (tile - __ldg(a.tile_off + lo)) * (2 * kRows);
-    const int32_t re = __ldg(a.offsets + lo + 1);
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      it.row_start[t] = rs + t * kRows;
-      it.nrows[t] = max(0, min(kRows, re - it.row_start[t]));
-      it.diag[t] = 1 << 30;
-      it.q0[t] = 0;
-      it.h[t] = 0;
-    }
-    it.key0 = seq_start(g, it.s) + b * g.bs;
-    it.nchunks = g.bs / kBN;
-  } else {
-    const int per_blk = g.bs / kRows;
-    if (a.own_head_pairs) {
-      const int hp_n = g.Hq / 2;
-      const int64_t inner = (int64_t)g.MB * g.num_seqs * hp_n;
-      const int qt = per_blk - 1 - (int)(item / inner);
-      int64_t rest = item % inner;
-      const int hp = (int)(rest % hp_n);
-      rest /= hp_n;
-      it.s = (int)(rest % g.num_seqs);
-      it.i_blk = (int)(rest / g.num_seqs);
-      const int32_t ts = seq_start(g, it.s), te = seq_end(g, it.s);
-      const int32_t q0 = ts + it.i_blk * g.bs + qt * kRows;
-      it.valid = q0 < te;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        it.h[t] = 2 * hp + t;
-        it.q0[t] = q0;
-        it.nrows[t] = max(0, min(kRows, te - q0));
-        it.diag[t] = qt;
-        it.row_start[t] = 0;
-      }
-      it.nchunks = qt + 1;
-      it.key0 = ts + it.i_blk * g.bs;
-    } else {
-      const int pairs = (per_blk + 1) / 2;
-      const int64_t inner = (int64_t)g.MB * g.num_seqs * g.Hq;
-      const int qp = pairs - 1 - (int)(item / inner);
-      int64_t rest = item % inner;
-      const int h = (int)(rest % g.Hq);
-      rest /= g.Hq;
-      it.s = (int)(rest % g.num_seqs);
-      it.i_blk = (int)(rest / g.num_seqs);
-      const int32_t ts = seq_start(g, it.s), te = seq_end(g, it.s);
-      const int32_t q0 = ts + it.i_blk * g.bs + 2 * qp * kRows;
-      it.valid = q0 < te;
-      const int qt1 = 2 * qp + 1;
-      const bool has1 = qt1 < per_blk && q0 + kRows < te;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        it.h[t] = h;
-        it.q0[t] = q0 + t * kRows;
-        it.nrows[t] = (t == 0 || has1) ? max(0, min(kRows, te - it.q0[t])) : 0;
-        it.diag[t] = 2 * qp + t;
-        it.row_start[t] = 0;
-      }
-      it.nchunks = has1 ? qt1 + 1 : 2 * qp + 1;
-      it.key0 = ts + it.i_blk * g.bs;
-    }
-    it.gk = it.h[0] / g.G;
-  }
-  return it;
-}
-
-// First valid item of this CTA at or after `item` (n when none is left).
-template <bool kOwn>
-__device__ __forceinline__ int64_t next_valid(const AttnArgs& a, int64_t item, int64_t n, Item& it) {
-  for (; item < n; item += gridDim.x) {
-    it = decode_item<kOwn>(a, item);
-    if (it.valid) return item;
-  }
-  return n;
-}
-
-// Q row of row r of tile t (-1 for padding rows); e receives the partial id (past mode).
-template <bool kOwn>
-__device__ __forceinline__ int64_t item_qrow(const AttnArgs& a, const Item& it, int t, int r, int32_t& e) {
-  e = -1;
-  if (r >= it.nrows[t]) return -1;
-  if constexpr (!kOwn) {
-    e = __ldg(a.rows + it.row_start[t] + r);
-    return e / (a.g.k - 1);
-  } else {
-    return (int64_t)(it.q0[t] + r) * a.g.Hq + it.h[t];
-  }
-}
-
-// cp.async of one Q row into tile t's 128-byte-swizzled buffer (zeros for padding rows).
-template <int D>
-__device__ __forceinline__ void gather_q_row(uint8_t* smem, int t, int r, const __nv_bfloat16* Q, int64_t qrow) {
-  using L = Layout<D>;
-  const __nv_bfloat16* src = qrow >= 0 ? Q + qrow * D : Q;
-  const uint32_t nb = qrow >= 0 ? 16u : 0u;
-  const uint32_t sQ = smem_u32(smem + L::kQ + t * L::kTile);
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) cp_async_16(sQ + sw128_offset(r, c, kRows), src + c * 8, nb);
-}
 
 template <int D, bool kOwn>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -235,8 +96,73 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kNumBars * 8);
   const Geom& g = a.g;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t n_items = num_items<kOwn>(a);
-  if ((int64_t)blockIdx.x >= n_items) return;
+
+  // ------------------------------------------------------------- work item
+  int gk, s, i_blk = 0, nchunks;
+  int32_t key0;
+  TileInfo ti[2];
+  if constexpr (!kOwn) {
+    const int32_t total = __ldg(a.tile_off + g.nbk);
+    const int32_t tile = (int32_t)blockIdx.x;
+    if (tile >= total) return;
+    int64_t lo = 0, hi = g.nbk - 1;  // last bucket whose first tile is <= tile
+    while (lo < hi) {
+      const int64_t mid = (lo + hi + 1) >> 1;
+      if (__ldg(a.tile_off + mid) <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int32_t b = (int32_t)(lo % g.MB);
+    s = (int)((lo / g.MB) % g.num_seqs);
+    gk = (int)(lo / ((int64_t)g.MB * g.num_seqs));
+    const int32_t rs = __ldg(a.offsets + lo) + (tile - __ldg(a.tile_off + lo)) * (2 * kRows);
+    const int32_t re = __ldg(a.offsets + lo + 1);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      ti[t].row_start = rs + t * kRows;
+      ti[t].nrows = max(0, min(kRows, re - ti[t].row_start));
+      ti[t].diag = 1 << 30;
+      ti[t].qrow_base = 0; ti[t].q0 = 0; ti[t].h = 0;
+    }
+    key0 = seq_start(g, s) + b * g.bs;
+    nchunks = g.bs / kBN;
+  } else {
+    const int per_blk = g.bs / kRows;
+    s = blockIdx.y;
+    const int32_t ts = seq_start(g, s), te = seq_end(g, s);
+    if (a.own_head_pairs) {
+      i_blk = blockIdx.x / per_blk;
+      const int qt = blockIdx.x - i_blk * per_blk;
+      const int32_t q0 = ts + i_blk * g.bs + qt * kRows;
+      if (q0 >= te) return;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        ti[t].h = 2 * blockIdx.z + t;
+        ti[t].q0 = q0;
+        ti[t].nrows = min(kRows, te - q0);
+        ti[t].diag = qt;
+        ti[t].row_start = 0;
+      }
+      nchunks = qt + 1;
+    } else {
+      const int pairs = (per_blk + 1) / 2;
+      i_blk = blockIdx.x / pairs;
+      const int qp = blockIdx.x - i_blk * pairs;
+      const int32_t q0 = ts + i_blk * g.bs + 2 * qp * kRows;
+      if (q0 >= te) return;
+      const int qt1 = 2 * qp + 1;
+      const bool has1 = qt1 < per_blk && q0 + kRows < te;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        ti[t].h = blockIdx.z;
+        ti[t].q0 = q0 + t * kRows;
+        ti[t].nrows = (t == 0 || has1) ? max(0, min(kRows, te - ti[t].q0)) : 0;
+        ti[t].diag = 2 * qp + t;
+        ti[t].row_start = 0;
+      }
+      nchunks = has1 ? qt1 + 1 : 2 * qp + 1;
+    }
+    gk = ti[0].h / g.G;
+    key0 = ts + i_blk * g.bs;
+  }
 
   // ------------------------------------------------------------- setup
   if (warp == 9) {
@@ -245,8 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
   }
   if (tid == 0) {
+    mbar_init(&bars[kQFull], 2 * kRows);
     for (int q = 0; q < 2; ++q) {
-      mbar_init(&bars[kQFull0 + q], kRows);
       mbar_init(&bars[kKFull0 + q], 1);
       mbar_init(&bars[kKEmpty0 + q], 1);
       mbar_init(&bars[kVFull0 + q], 1);
@@ -268,125 +194,118 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ========================================================= softmax warpgroups
     const int t = warp >> 2;           // tile
     const int r = tid & (kRows - 1);   // row = TMEM lane
+    const TileInfo& T_ = ti[t];
+    int64_t qrow = -1;
+    int32_t e = -1;
+    if (r < T_.nrows) {
+      if constexpr (!kOwn) {
+        e = __ldg(a.rows + T_.row_start + r);
+        qrow = e / (g.k - 1);
+      } else {
+        qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
+      }
+    }
+    {  // gather this row of Q into tile t (zeros for padding rows)
+      const __nv_bfloat16* src = qrow >= 0 ? a.Q + qrow * D : a.Q;
+      const uint32_t nb = qrow >= 0 ? 16u : 0u;
+      const uint32_t sQ = smem_u32(smem + L::kQ + t * L::kTile);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) cp_async_16(sQ + sw128_offset(r, c, kRows), src + c * 8, nb);
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[kQFull]);
+    }
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + kColS + t * kBN;
     const uint32_t tP = tS + kColP;
     const uint32_t tO = tmem + lane_off + kColO + t * 128;
     const float c2 = g.scale_log2;
-    Item cur, nxt;
-    int64_t item = next_valid<kOwn>(a, blockIdx.x, n_items, cur);
-    int32_t e = -1;
-    int64_t qrow = -1;
-    if (item < n_items) {
-      qrow = item_qrow<kOwn>(a, cur, t, r, e);
-      gather_q_row<D>(smem, t, r, a.Q, qrow);
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(&bars[kQFull0 + t]);
-    }
-    uint32_t gc = 0, ic = 0;  // chunks and items processed so far (barrier phases)
-    while (item < n_items && ok) {
-      const int64_t item_n = next_valid<kOwn>(a, item + gridDim.x, n_items, nxt);
-      int32_t e_n = -1;
-      const int64_t qrow_n = item_n < n_items ? item_qrow<kOwn>(a, nxt, t, r, e_n) : -1;
-      const int nch = cur.nchunks;
-      const int diag = cur.diag[t];
-      float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < nch && ok; ++j) {
-        const uint32_t gj = gc + j;
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull0 + t], gj & 1, g.err));
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
-        tmem_wait_ld();
-        // this item's last S of this tile has been read, so the tile's Q buffer is free: gather
-        // the next item's rows while the softmax and the epilogue run
-        if (j == nch - 1 && item_n < n_items) gather_q_row<D>(smem, t, r, a.Q, qrow_n);
-        // scaled-logit row max (log2 units); the causal mask applies to the diagonal chunk
-        // only (in the query-tile-pair layout, chunks after a tile's diagonal are all masked)
-        const bool masked = kOwn && j >= diag;
-        const int lim = (kOwn && j == diag) ? r + 1 : (masked ? 0 : kBN);
-        float mv[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mv[q] = -INFINITY;
-        if (!masked) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int x = 0; x < 32; ++x) mv[x & 7] = fmaxf(mv[x & 7], __uint_as_float(sr[c][x]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int x = 0; x < 32; ++x)
-              if (c * 32 + x < lim) mv[x & 7] = fmaxf(mv[x & 7], __uint_as_float(sr[c][x]));
-        }
-        float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])), fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
-        mx *= c2;
-        // running max: rescale the TMEM accumulator only when it grows by more than 2^8
-        // (p <= 256 otherwise, harmless in fp32 sums and bf16 P).  The previous PV of this
-        // tile has completed here: the MMA that produced this S was issued after it.
-        if (j == 0) {
-          m = mx;
-        } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
-          const float m_new = fmaxf(m, mx);
-          const float alpha = ex2(m - m_new);
-          l *= alpha;
-          m = m_new;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(tO + c * 32, o);
-          }
-        }
-        // p = 2^(s*c2 - m); P (bf16 pairs) overwrites the first 64 S columns (S is in registers)
-        float rv[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) rv[q] = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int c = 2 * cc + h2;
-#pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              float p0 = ex2(fmaf(__uint_as_float(sr[c][x]), c2, -m));
-              float p1 = ex2(fmaf(__uint_as_float(sr[c][x + 1]), c2, -m));
-              if (masked) {
-                if (c * 32 + x >= lim) p0 = 0.f;
-                if (c * 32 + x + 1 >= lim) p1 = 0.f;
-              }
-              rv[x & 7] += p0;
-              rv[(x & 7) + 1] += p1;
-              pk[16 * h2 + (x >> 1)] = pack_bf16x2(p0, p1);
-            }
-          }
-          tmem_st32(tP + cc * 32, pk);
-        }
-        l += ((rv[0] + rv[1]) + (rv[2] + rv[3])) + ((rv[4] + rv[5]) + (rv[6] + rv[7]));
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars[kPFull0 + t]);
-      }
-      if (!ok) break;
-      // hand the next item's Q tile to the MMA warp before this item's epilogue
-      if (item_n < n_items) {
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(&bars[kQFull0 + t]);
-      }
-      // ------------------------------------------------------- epilogue of this item
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull0 + t], ic & 1, g.err));
+    float m = -INFINITY, l = 0.f;
+    for (int j = 0; j < nchunks && ok; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull0 + t], j & 1, g.err));
       if (!ok) break;
       tc_fence_after();
-      const int nrows = cur.nrows[t];
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+      tmem_wait_ld();
+      // scaled-logit row max (log2 units); the causal mask applies to the diagonal chunk only
+      // (keys after the diagonal chunk, in the query-tile-pair layout, are all masked)
+      const bool masked = kOwn && j >= T_.diag;
+      const int lim = (kOwn && j == T_.diag) ? r + 1 : (masked ? 0 : kBN);
+      // eight independent running maxima keep the dependency chain short
+      float mv[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mv[q] = -INFINITY;
+      if (!masked) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int x = 0; x < 32; ++x) mv[x & 7] = fmaxf(mv[x & 7], __uint_as_float(sr[c][x]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            if (c * 32 + x < lim) mv[x & 7] = fmaxf(mv[x & 7], __uint_as_float(sr[c][x]));
+      }
+      float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])), fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+      mx *= c2;
+      // running max: rescale the TMEM accumulator only when it grows by more than 2^8
+      // (p <= 256 otherwise, harmless in fp32 sums and bf16 P).  At this point the previous
+      // PV of this tile has completed: the MMA that produced this S was issued after it.
+      if (j == 0) {
+        m = mx;
+      } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
+        const float m_new = fmaxf(m, mx);
+        const float alpha = ex2(m - m_new);
+        l *= alpha;
+        m = m_new;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+          tmem_st32(tO + c * 32, o);
+        }
+      }
+      // p = 2^(s*c2 - m); P (bf16 pairs) overwrites the first 64 S columns (S is in registers)
+      float rv[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) rv[q] = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int c = 2 * cc + h2;
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            float p0 = ex2(fmaf(__uint_as_float(sr[c][x]), c2, -m));
+            float p1 = ex2(fmaf(__uint_as_float(sr[c][x + 1]), c2, -m));
+            if (masked) {
+              if (c * 32 + x >= lim) p0 = 0.f;
+              if (c * 32 + x + 1 >= lim) p1 = 0.f;
+            }
+            rv[x & 7] += p0;
+            rv[(x & 7) + 1] += p1;
+            pk[16 * h2 + (x >> 1)] = pack_bf16x2(p0, p1);
+          }
+        }
+        tmem_st32(tP + cc * 32, pk);
+      }
+      const float rs = ((rv[0] + rv[1]) + (rv[2] + rv[3])) + ((rv[4] + rv[5]) + (rv[6] + rv[7]));
+      l += rs;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars[kPFull0 + t]);
+    }
+    // ------------------------------------------------------- epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[kOFull0 + t], 0, g.err));
+    if (ok) {
+      tc_fence_after();
       const float inv_l = 1.f / l;
       const float lse_row = (m + __log2f(l)) * kLn2;
       if constexpr (!kOwn) {
@@ -395,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t o[32];
           tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
-          if (r < nrows) {
+          if (r < T_.nrows) {
             float4* dst = reinterpret_cast<float4*>(a.part_o + (int64_t)e * D + c * 32);
 #pragma unroll
             for (int x = 0; x < 32; x += 4)
@@ -403,17 +322,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         __uint_as_float(o[x + 2]) * inv_l, __uint_as_float(o[x + 3]) * inv_l);
           }
         }
-        if (r < nrows) a.part_lse[e] = lse_row;
+        if (r < T_.nrows) a.part_lse[e] = lse_row;
       } else {
         // online-softmax merge of the own-block result with the row's past partials
         float M = lse_row;
         int32_t pe[kMaxTopK];
         float pl[kMaxTopK];
         int np = 0;
-        if (r < nrows) {
+        if (r < T_.nrows) {
           for (int slot = 1; slot < g.k; ++slot) {
             const int32_t b = __ldg(a.sel + qrow * g.k + slot);
-            if (b >= 0 && b < cur.i_blk) {
+            if (b >= 0 && b < i_blk) {
               pe[np] = (int32_t)(qrow * (g.k - 1) + slot - 1);
               pl[np] = __ldg(a.part_lse + pe[np]);
               M = fmaxf(M, pl[np]);
@@ -434,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t o[32];
           tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
-          if (r < nrows) {
+          if (r < T_.nrows) {
             float acc[32];
 #pragma unroll
             for (int x = 0; x < 32; ++x) acc[x] = __uint_as_float(o[x]) * a_self;
@@ -457,47 +376,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        pack_bf16x2(acc[x + 4], acc[x + 5]), pack_bf16x2(acc[x + 6], acc[x + 7]));
           }
         }
-        if (r < nrows) a.LSE[qrow] = M + __logf(sumw);
+        if (r < T_.nrows) a.LSE[qrow] = M + __logf(sumw);
       }
-      // The O reads above complete (wait::ld) before this warpgroup's next arrival on its P
-      // barrier, which the next item's first PV (which overwrites O) waits for.
-      gc += nch;
-      ++ic;
-      item = item_n;
-      cur = nxt;
-      qrow = qrow_n;
-      e = e_n;
     }
   } else if (warp == 8) {
     // ========================================================= TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      uint32_t gc = 0;
-      Item it;
-      for (int64_t item = next_valid<kOwn>(a, blockIdx.x, n_items, it); item < n_items && ok;
-           item = next_valid<kOwn>(a, item + gridDim.x, n_items, it)) {
-        for (int j = 0; j < it.nchunks && ok; ++j) {
-          const uint32_t gj = gc + j;
-          const int st = gj & 1;
-          const uint32_t u = gj >> 1;
-          const int tok = it.key0 + j * kBN;
-          if (u > 0) ok = mbar_wait(&bars[kKEmpty0 + st], (u - 1) & 1, g.err);
-          if (!ok) break;
-          mbar_expect_tx(&bars[kKFull0 + st], L::kTile);
+      for (int j = 0; j < nchunks && ok; ++j) {
+        const int st = j & 1, u = j >> 1;
+        const int tok = key0 + j * kBN;
+        if (u > 0) ok = mbar_wait(&bars[kKEmpty0 + st], (u - 1) & 1, g.err);
+        if (!ok) break;
+        mbar_expect_tx(&bars[kKFull0 + st], L::kTile);
 #pragma unroll
-          for (int hh = 0; hh < D / 64; ++hh)
-            tma_load_3d(smem + L::kK0 + st * L::kTile + hh * kRows * 128, &tmK, &bars[kKFull0 + st], hh * 64,
-                        it.gk, tok);
-          if (u > 0) ok = mbar_wait(&bars[kVEmpty0 + st], (u - 1) & 1, g.err);
-          if (!ok) break;
-          mbar_expect_tx(&bars[kVFull0 + st], L::kTile);
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_3d(smem + L::kK0 + st * L::kTile + hh * kRows * 128, &tmK, &bars[kKFull0 + st], hh * 64, gk, tok);
+        if (u > 0) ok = mbar_wait(&bars[kVEmpty0 + st], (u - 1) & 1, g.err);
+        if (!ok) break;
+        mbar_expect_tx(&bars[kVFull0 + st], L::kTile);
 #pragma unroll
-          for (int hh = 0; hh < D / 64; ++hh)
-            tma_load_3d(smem + L::kV0 + st * L::kTile + hh * kRows * 128, &tmV, &bars[kVFull0 + st], hh * 64,
-                        it.gk, tok);
-        }
-        gc += it.nchunks;
+        for (int hh = 0; hh < D / 64; ++hh)
+          tma_load_3d(smem + L::kV0 + st * L::kTile + hh * kRows * 128, &tmV, &bars[kVFull0 + st], hh * 64, gk, tok);
       }
     }
   } else if (warp == 9) {
@@ -508,8 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sQ = smem_u32(smem + L::kQ);
       const uint32_t sK0 = smem_u32(smem + L::kK0);
       const uint32_t sV0 = smem_u32(smem + L::kV0);
-      auto issue_s = [&](int t, uint32_t gj) {
-        const uint32_t qb = sQ + t * L::kTile, kb = sK0 + (gj & 1) * L::kTile;
+      auto issue_s = [&](int t, int j) {
+        const uint32_t qb = sQ + t * L::kTile, kb = sK0 + (j & 1) * L::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
@@ -518,57 +419,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bars[kSFull0 + t]);
       };
-      auto issue_pv = [&](int t, uint32_t gj, bool first) {
-        const uint32_t vb = sV0 + (gj & 1) * L::kTile;
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t vb = sV0 + (j & 1) * L::kTile;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
           mma_bf16_ts(tmem + kColO + t * 128, tmem + kColS + t * kBN + kColP + kk * 8,
-                      sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), idO, (!first || kk > 0) ? 1u : 0u);
+                      sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
       };
-      uint32_t gc = 0, ic = 0;
-      Item it;
-      for (int64_t item = next_valid<kOwn>(a, blockIdx.x, n_items, it); item < n_items && ok;
-           item = next_valid<kOwn>(a, item + gridDim.x, n_items, it)) {
-        const int nch = it.nchunks;
-        ok = mbar_wait(&bars[kQFull0], ic & 1, g.err) && mbar_wait(&bars[kKFull0 + (gc & 1)], (gc >> 1) & 1, g.err);
-        if (!ok) break;
+      ok = mbar_wait(&bars[kQFull], 0, g.err) && mbar_wait(&bars[kKFull0], 0, g.err);
+      if (ok) {
         tc_fence_after();
-        issue_s(0, gc);
-        ok = mbar_wait(&bars[kQFull1], ic & 1, g.err);
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(1, gc);
-        mma_commit(&bars[kKEmpty0 + (gc & 1)]);
-        for (int j = 0; j < nch && ok; ++j) {
-          const uint32_t gj = gc + j;
-          const bool more = j + 1 < nch;
-          ok = mbar_wait(&bars[kVFull0 + (gj & 1)], (gj >> 1) & 1, g.err) &&
-               mbar_wait(&bars[kPFull0], gj & 1, g.err);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(0, gj, j == 0);
-          if (!more) mma_commit(&bars[kOFull0]);
-          if (more) {
-            ok = mbar_wait(&bars[kKFull0 + ((gj + 1) & 1)], ((gj + 1) >> 1) & 1, g.err);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(0, gj + 1);
-          }
-          ok = mbar_wait(&bars[kPFull1], gj & 1, g.err);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(1, gj, j == 0);
-          mma_commit(&bars[kVEmpty0 + (gj & 1)]);
-          if (!more) mma_commit(&bars[kOFull1]);
-          if (more) {
-            issue_s(1, gj + 1);
-            mma_commit(&bars[kKEmpty0 + ((gj + 1) & 1)]);
-          }
-        }
-        gc += nch;
-        ++ic;
+        issue_s(0, 0);
+        issue_s(1, 0);
+        mma_commit(&bars[kKEmpty0]);
       }
-      // every MMA issued above has completed once kDone fires
+      for (int j = 0; j < nchunks && ok; ++j) {
+        const bool more = j + 1 < nchunks;
+        ok = mbar_wait(&bars[kVFull0 + (j & 1)], (j >> 1) & 1, g.err) && mbar_wait(&bars[kPFull0], j & 1, g.err);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (!more) mma_commit(&bars[kOFull0]);
+        if (more) {
+          ok = mbar_wait(&bars[kKFull0 + ((j + 1) & 1)], ((j + 1) >> 1) & 1, g.err);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        ok = mbar_wait(&bars[kPFull1], j & 1, g.err);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        mma_commit(&bars[kVEmpty0 + (j & 1)]);
+        if (!more) mma_commit(&bars[kOFull1]);
+        if (more) {
+          issue_s(1, j + 1);
+          mma_commit(&bars[kKEmpty0 + ((j + 1) & 1)]);
+        }
+      }
       mma_commit(&bars[kDone]);
       mbar_wait(&bars[kDone], 0, g.err);
     }
@@ -582,29 +470,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-int sm_count() {
-  static int n = 0;
-  if (n <= 0) {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-        v > 0)
-      n = v;
-    else
-      n = 148;
-  }
-  return n;
-}
-
 template <int D, bool kOwn>
 cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
-                      const int32_t* sel, const Work& w, __nv_bfloat16* O, float* LSE, int64_t max_items,
-                      int head_pairs, int64_t own_items, cudaStream_t st) {
+                      const int32_t* sel, const Work& w, __nv_bfloat16* O, float* LSE, dim3 grid, int head_pairs,
+                      cudaStream_t st) {
   CUtensorMap tk, tv;
   cudaError_t e = make_rows_map(&tk, K, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
   e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
-  AttnArgs a{g, Q, sel, w.offsets, w.tile_off, w.rows, w.part_o, w.part_lse, O, LSE, head_pairs, own_items};
+  AttnArgs a{g, Q, sel, w.offsets, w.tile_off, w.rows, w.part_o, w.part_lse, O, LSE, head_pairs};
   const int smem = Layout<D>::kAlloc;
   e = cudaFuncSetAttribute(attn_tc_kernel<D, kOwn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -613,10 +488,7 @@ cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16
   e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D, kOwn>);
   if (e != cudaSuccess) return e;
   if ((uint32_t)fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
-  // persistent: one CTA per SM (its shared memory and 512 TMEM columns allow no second one)
-  const int64_t grid = max_items < sm_count() ? max_items : sm_count();
-  if (grid <= 0) return cudaSuccess;
-  attn_tc_kernel<D, kOwn><<<(unsigned)grid, kThreads, smem, st>>>(tk, tv, a);
+  attn_tc_kernel<D, kOwn><<<grid, kThreads, smem, st>>>(tk, tv, a);
   return cudaGetLastError();
 }
 
@@ -626,8 +498,9 @@ cudaError_t launch_attn_past(const Geom& g, const __nv_bfloat16* Q, const __nv_b
                              const __nv_bfloat16* V, const Work& w, cudaStream_t st) {
   if (g.T == 0 || g.k < 2 || g.R == 0) return cudaSuccess;
   const int64_t tiles = (g.R + kPastTileRows - 1) / kPastTileRows + g.nbk;  // bound on routed tile pairs
-  if (g.D == 64) return launch_tc<64, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, tiles, 0, 0, st);
-  return launch_tc<128, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, tiles, 0, 0, st);
+  dim3 grid((unsigned)tiles);
+  if (g.D == 64) return launch_tc<64, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, grid, 0, st);
+  return launch_tc<128, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, grid, 0, st);
 }
 
 cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
@@ -636,10 +509,10 @@ cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_b
   if (g.T == 0) return cudaSuccess;
   const int per_blk = g.bs / kRows;
   const int head_pairs = (g.G % 2 == 0) ? 1 : 0;
-  const int64_t items = head_pairs ? (int64_t)per_blk * g.MB * g.num_seqs * (g.Hq / 2)
-                                   : (int64_t)((per_blk + 1) / 2) * g.MB * g.num_seqs * g.Hq;
-  if (g.D == 64) return launch_tc<64, true>(g, Q, K, V, sel, w, O, LSE, items, head_pairs, items, st);
-  return launch_tc<128, true>(g, Q, K, V, sel, w, O, LSE, items, head_pairs, items, st);
+  dim3 grid = head_pairs ? dim3((unsigned)(g.MB * per_blk), (unsigned)g.num_seqs, (unsigned)(g.Hq / 2))
+                         : dim3((unsigned)(g.MB * ((per_blk + 1) / 2)), (unsigned)g.num_seqs, (unsigned)g.Hq);
+  if (g.D == 64) return launch_tc<64, true>(g, Q, K, V, sel, w, O, LSE, grid, head_pairs, st);
+  return launch_tc<128, true>(g, Q, K, V, sel, w, O, LSE, grid, head_pairs, st);
 }
 
 int launches_per_forward(const Geom& g) {
