@@ -308,34 +308,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const float lse_row = (m + __log2f(l)) * kLn2;
-      if constexpr (!kOwn) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-          if (r < T_.nrows) {
-            float4* dst = reinterpret_cast<float4*>(a.part_o + (int64_t)e * D + c * 32);
-#pragma unroll
-            for (int x = 0; x < 32; x += 4)
-              dst[x >> 2] = make_float4(__uint_as_float(o[x]) * inv_l, __uint_as_float(o[x + 1]) * inv_l,
-                                        __uint_as_float(o[x + 2]) * inv_l, __uint_as_float(o[x + 3]) * inv_l);
-          }
-        }
-        if (r < T_.nrows) a.part_lse[e] = lse_row;
-      } else {
-        // online-softmax merge of the own-block result with the row's past partials
-        float M = lse_row;
-        int32_t pe[kMaxTopK];
-        float pl[kMaxTopK];
-        int np = 0;
+      // Each warp stages its 32 rows (fp32, D columns) in shared memory that no MMA reads any
+      // more (this tile's Q buffer and one K stage: every QK^T MMA completed before the O
+      // barrier fired), then writes whole rows with coalesced stores.  16-byte chunks of a
+      // staged row are XOR-swizzled by (row mod 8) to spread the row-per-thread writes over
+      // the banks.
+      const int wq = warp & 3;
+      float* stg = reinterpret_cast<float*>(smem + (wq < 2 ? L::kQ : L::kK0) + t * L::kTile + (wq & 1) * (L::kTile / 2));
+      auto stg_at = [&](int row, int col) -> float* {
+        return stg + row * D + ((((col >> 2) ^ (row & 7)) << 2) | (col & 3));
+      };
+      float scale_row = inv_l;
+      // own mode: merge weights of this row (own block and its past partials)
+      float M = lse_row, inv_w = 1.f;
+      int32_t pe[kMaxTopK];
+      float pw[kMaxTopK];
+      int np = 0;
+      if constexpr (kOwn) {
         if (r < T_.nrows) {
           for (int slot = 1; slot < g.k; ++slot) {
             const int32_t b = __ldg(a.sel + qrow * g.k + slot);
             if (b >= 0 && b < i_blk) {
               pe[np] = (int32_t)(qrow * (g.k - 1) + slot - 1);
-              pl[np] = __ldg(a.part_lse + pe[np]);
-              M = fmaxf(M, pl[np]);
+              pw[np] = __ldg(a.part_lse + pe[np]);
+              M = fmaxf(M, pw[np]);
               ++np;
             }
           }
@@ -343,40 +339,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float w_self = __expf(lse_row - M);
         float sumw = w_self;
         for (int q = 0; q < np; ++q) {
-          pl[q] = __expf(pl[q] - M);
-          sumw += pl[q];
+          pw[q] = __expf(pw[q] - M);
+          sumw += pw[q];
         }
-        const float inv_w = 1.f / sumw;
-        const float a_self = w_self * inv_l * inv_w;
+        inv_w = 1.f / sumw;
+        for (int q = 0; q < np; ++q) pw[q] *= inv_w;
+        scale_row = w_self * inv_l * inv_w;
+        if (r < T_.nrows) a.LSE[qrow] = M + __logf(sumw);
+      } else {
+        if (r < T_.nrows) a.part_lse[e] = lse_row;
+      }
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-          if (r < T_.nrows) {
-            float acc[32];
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 32; ++x) acc[x] = __uint_as_float(o[x]) * a_self;
-            for (int q = 0; q < np; ++q) {
-              const float4* src = reinterpret_cast<const float4*>(a.part_o + (int64_t)pe[q] * D + c * 32);
-              const float wq = pl[q] * inv_w;
+        for (int x = 0; x < 32; x += 4)
+          *reinterpret_cast<float4*>(stg_at(lane, c * 32 + x)) =
+              make_float4(__uint_as_float(o[x]) * scale_row, __uint_as_float(o[x + 1]) * scale_row,
+                          __uint_as_float(o[x + 2]) * scale_row, __uint_as_float(o[x + 3]) * scale_row);
+      }
+      __syncwarp();
+      if constexpr (!kOwn) {
+        for (int rr = 0; rr < 32; ++rr) {
+          const int32_t er = __shfl_sync(0xffffffffu, e, rr);
+          if (er < 0) continue;
+          float* dst = a.part_o + (int64_t)er * D + lane;
 #pragma unroll
-              for (int x = 0; x < 32; x += 4) {
-                const float4 v = __ldg(src + (x >> 2));
-                acc[x] = fmaf(wq, v.x, acc[x]);
-                acc[x + 1] = fmaf(wq, v.y, acc[x + 1]);
-                acc[x + 2] = fmaf(wq, v.z, acc[x + 2]);
-                acc[x + 3] = fmaf(wq, v.w, acc[x + 3]);
-              }
+          for (int c = 0; c < D / 32; ++c) dst[c * 32] = *stg_at(rr, c * 32 + lane);
+        }
+      } else {
+        // eight rows at a time, so their partial rows are all in flight together
+        constexpr int kU = 8;
+        for (int rr0 = 0; rr0 < 32; rr0 += kU) {
+          int64_t qr[kU];
+          int npr[kU];
+          float acc[kU][D / 32];
+          int npmax = 0;
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            qr[u] = __shfl_sync(0xffffffffu, qrow, rr0 + u);
+            npr[u] = __shfl_sync(0xffffffffu, np, rr0 + u);
+            npmax = max(npmax, npr[u]);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) acc[u][c] = *stg_at(rr0 + u, c * 32 + lane);
+          }
+          for (int q = 0; q < npmax; ++q) {
+            float tmp[kU][D / 32];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+              const int32_t pq = __shfl_sync(0xffffffffu, pe[q], rr0 + u);
+              const float* src = a.part_o + (int64_t)pq * D + lane;
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) tmp[u][c] = q < npr[u] ? __ldg(src + c * 32) : 0.f;
             }
-            uint4* dst = reinterpret_cast<uint4*>(a.O + qrow * D + c * 32);
 #pragma unroll
-            for (int x = 0; x < 32; x += 8)
-              dst[x >> 3] = make_uint4(pack_bf16x2(acc[x], acc[x + 1]), pack_bf16x2(acc[x + 2], acc[x + 3]),
-                                       pack_bf16x2(acc[x + 4], acc[x + 5]), pack_bf16x2(acc[x + 6], acc[x + 7]));
+            for (int u = 0; u < kU; ++u) {
+              const float wgt = __shfl_sync(0xffffffffu, pw[q], rr0 + u);
+              if (q < npr[u])
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) acc[u][c] = fmaf(wgt, tmp[u][c], acc[u][c]);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            if (qr[u] < 0) continue;
+            __nv_bfloat16* dst = a.O + qr[u] * D + lane;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) dst[c * 32] = __float2bfloat16_rn(acc[u][c]);
           }
         }
-        if (r < T_.nrows) a.LSE[qrow] = M + __logf(sumw);
       }
     }
   } else if (warp == 8) {
