@@ -125,13 +125,28 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def make_host_inputs(w: synth.Workload, pinned: bool):
+def max_over_ranks(value: float, dist, device=None) -> float:
+    """Largest value over all ranks (the job's time is its slowest rank's time)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, steps: int, max_ms: float) -> float:
+    """Units all ranks processed over the timed region, per second of its slowest rank."""
+    return units_per_rank * world * steps / (max_ms / 1e3)
+
+
+def make_host_inputs(w: synth.Workload, pinned: bool, nthreads: int | None = None):
     import torch
     out = {}
     for which in ("q", "k", "v"):
         shape = (w.total_tokens, w.heads(which), w.head_dim)
         t = torch.empty(shape, dtype=torch.int16, pin_memory=pinned)
-        w.fill(which, out=t.numpy().view(np.uint16))
+        w.fill(which, out=t.numpy().view(np.uint16), nthreads=nthreads)
         out[which] = t.view(torch.bfloat16)
     return out
 
@@ -180,7 +195,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    host = make_host_inputs(w, pinned=True)
+    host = make_host_inputs(w, pinned=True, nthreads=max(1, (os.cpu_count() or 1) // world))
     Q = host["q"].to(dev, non_blocking=True)
     K = host["k"].to(dev, non_blocking=True)
     V = host["v"].to(dev, non_blocking=True)
@@ -226,16 +241,12 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
     clk = clocks.stop()
     total_ms = evs[0][0].elapsed_time(evs[-1][5])
     stage_ms = {s: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j, s in enumerate(stages)}
-    t_max = total_ms
-    if dist is not None:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
+    t_max = max_over_ranks(total_ms, dist, dev)
     routed = int((sel[:, :, 1:] >= 0).sum().item()) if w.top_k > 1 else 0
     # sel slot >= 1 is valid exactly when it names a past block; verify the count from the rows
     fl = flop_counts(w, routed)
     ms_step = t_max / args.steps
-    tokens_per_s = T * world * args.steps / (t_max / 1e3)
+    tokens_per_s = job_throughput(T, world, args.steps, t_max)
 
     # ----- end to end through the public call with host buffers (pinned), copies timed
     e2e = None
@@ -262,14 +273,10 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = a.elapsed_time(b)
-        if dist is not None:
-            tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(a.elapsed_time(b), dist, dev)
         h2d = sum(host[x].numel() * 2 for x in ("q", "k", "v"))
         d2h = O.numel() * 2 + LSE.numel() * 4
-        e2e = {"value": T * world * n_e2e / (e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": job_throughput(T, world, n_e2e, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
 
     peaks, peak_kind = load_peaks()

@@ -25,7 +25,7 @@ STATUS = {0: "MOBA_OK", 1: "MOBA_ERR_INVALID_ARG", 2: "MOBA_ERR_UNSUPPORTED",
 EXPORTS = ("moba_kbar_elems", "moba_workspace_size", "moba_pool_keys", "moba_gate_topk",
            "moba_attn_fwd", "moba_fwd", "moba_route", "moba_attn_past", "moba_attn_self_merge",
            "moba_launches_per_forward", "moba_read_device_error", "moba_status_string",
-           "moba_last_error", "moba_gate_topk_noalloc")
+           "moba_last_error", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait")
 
 
 class MobaError(RuntimeError):
@@ -78,6 +78,8 @@ def load():
         for f in ("moba_pool_keys", "moba_gate_topk", "moba_attn_fwd", "moba_fwd", "moba_route",
                   "moba_attn_past", "moba_attn_self_merge"):
             getattr(lib, f).restype = ctypes.c_int
+        lib.moba_selftest_bounded_wait.argtypes = [ctypes.POINTER(ctypes.c_int32)]
+        lib.moba_selftest_bounded_wait.restype = ctypes.c_int
         lib.moba_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int]
         lib.moba_read_device_error.restype = ctypes.c_int
         lib.moba_status_string.argtypes = [ctypes.c_int]
@@ -210,6 +212,13 @@ def moba_read_device_error(clear: bool = False) -> int:
     """Device error word of the current device (non-zero: a kernel wait gave up)."""
     v = ctypes.c_int32(0)
     _check(load().moba_read_device_error(ctypes.byref(v), 1 if clear else 0))
+    return int(v.value)
+
+
+def moba_selftest_bounded_wait() -> int:
+    """Run the bounded-wait failure path once; returns the device error word it produced."""
+    v = ctypes.c_int32(0)
+    _check(load().moba_selftest_bounded_wait(ctypes.byref(v)))
     return int(v.value)
 
 

@@ -7,9 +7,21 @@
 
 #include "moba.h"
 #include "moba_internal.cuh"
+#include "sm100.cuh"
 
 // Device error word: kernels OR a code into it when a bounded wait gives up.
 __device__ int g_moba_device_error = 0;
+
+// One thread waits on an mbarrier phase that nothing completes, through the same bounded wait
+// the tensor-core kernels use: the wait gives up, sets the error word and the kernel returns.
+__global__ void bounded_wait_selftest_kernel(int* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    moba::mbar_init(&bar, 1);
+    moba::fence_mbar_init();
+    moba::mbar_wait(&bar, 0, err);
+  }
+}
 
 namespace {
 
@@ -349,6 +361,27 @@ const char* moba_status_string(int status) {
 }
 
 const char* moba_last_error(void) { return g_err; }
+
+moba_status moba_selftest_bounded_wait(int32_t* device_error) {
+  g_err[0] = 0;
+  if (!device_error) return fail(MOBA_ERR_INVALID_ARG, "device_error is NULL");
+  moba::Geom g;
+  MOBA_TRY(check_device(&g));
+  cudaError_t e = cudaMemset(g.err, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  bounded_wait_selftest_kernel<<<1, 32>>>(g.err);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test");
+  int v = 0;
+  e = cudaMemcpy(&v, g.err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  e = cudaMemset(g.err, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  *device_error = v;
+  return MOBA_OK;
+}
 
 moba_status moba_read_device_error(int32_t* value, int clear) {
   g_err[0] = 0;

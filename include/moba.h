@@ -181,6 +181,14 @@ MOBA_API int moba_launches_per_forward(const moba_params* p);
  */
 MOBA_API moba_status moba_read_device_error(int32_t* value, int clear);
 
+/*
+ * Exercises the failure path of those bounded waits: one thread waits on an mbarrier phase
+ * that nothing completes; after the wait limit (about 2 s) it gives up, sets the device error
+ * word and returns.  Synchronous.  *device_error receives the word's value (1 when the path
+ * works); the word is cleared before and after.
+ */
+MOBA_API moba_status moba_selftest_bounded_wait(int32_t* device_error);
+
 /* Static description of a status code. */
 MOBA_API const char* moba_status_string(int status);
 

@@ -28,6 +28,18 @@ SMALL = {
                                rope_theta=500000.0),
     # uniform batch expressed through cu_seqlens
     "batch3": synth.Workload("batch3", [1024, 1024, 1024], 2, 1, 64, 128, 3, seed=12),
+    # odd GQA group (G = 3): own-block tiles pair consecutive query tiles of one head
+    "gqa_odd": synth.Workload("gqa_odd", [1500, 640], 6, 2, 128, 256, 3, seed=13,
+                              rope_theta=500000.0, plant=0.5),
+    # empty sequences inside a packed batch
+    "empty_seqs": synth.Workload("empty_seqs", [300, 0, 700, 0, 129], 4, 2, 64, 128, 3, seed=14),
+    # the largest block size, one full block plus a partial one
+    "bs8192": synth.Workload("bs8192", [9000], 2, 1, 128, 8192, 2, seed=15, rope_theta=500000.0),
+    # the largest top_k with more blocks than it
+    "top16": synth.Workload("top16", [2560, 1100], 2, 2, 128, 128, 16, seed=16),
+    # many short sequences
+    "many_seqs": synth.Workload("many_seqs", list(np.random.default_rng(17).integers(1, 300, 300)), 2, 1, 64,
+                                128, 3, seed=17),
 }
 
 
