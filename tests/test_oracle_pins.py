@@ -315,3 +315,9 @@ def test_sampled_rows_equal_full_rows():
     r = oracle.rows(pr, w.rows("q", tok, hd), K, V, full["Kbar"], tok, hd)
     np.testing.assert_array_equal(r["sel"], full["sel"][tok, hd])
     np.testing.assert_array_equal(r["O"], full["O"][tok, hd])
+
+
+def test_bf16_ulp_helper_of_the_parity_rule():
+    from _harness import bf16_ulp
+    np.testing.assert_array_equal(bf16_ulp(np.array([1.0, 1.5, 2.0, 4.5, -0.3])),
+                                  [2.0 ** -7, 2.0 ** -7, 2.0 ** -6, 2.0 ** -5, 2.0 ** -9])
