@@ -125,6 +125,25 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def past_kernel_traffic(routed_rows: int):
+    """DRAM bytes per launch of the past-block attention kernel, from the committed ncu
+    record scaled by routed rows, or None when the kernel sources changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "attn_past_traffic.json")
+    if not os.path.exists(path):
+        return None, "no capture"
+    with open(path) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for name in rec["source_files"]:
+        with open(os.path.join(ROOT, name), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec["source_sha256"]:
+        return None, "kernel changed since the capture"
+    per_row = (rec["dram_bytes_read"] + rec["dram_bytes_write"]) / rec["routed_rows"]
+    return per_row * routed_rows, "scaled from the %s capture by routed rows" % rec["workload"]
+
+
 def max_over_ranks(value: float, dist, device=None) -> float:
     """Largest value over all ranks (the job's time is its slowest rank's time)."""
     if dist is None:
@@ -279,6 +298,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
         e2e = {"value": job_throughput(T, world, n_e2e, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
 
+    traffic, traffic_note = past_kernel_traffic(routed)
     peaks, peak_kind = load_peaks()
     peak_tf = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     past_s = stage_ms["past"] / 1e3
@@ -310,7 +330,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
         "roofline": {"bound": "tensor", "kernel": "past-block attention", "achieved": achieved,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
                      "peak_kind": "%s bf16 sustained (kernel timed inside a long step)" % peak_kind,
-                     "traffic": None},
+                     "traffic": traffic, "traffic_note": traffic_note},
         "clocks": clk,
         "gpu_launches": mb.moba_launches_per_forward(p) * args.steps,
         "e2e": e2e,
@@ -358,7 +378,7 @@ def run_reference(args, w: synth.Workload, rank: int) -> dict | None:
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", default="prefill1m", choices=sorted(synth.CONFIGS))
