@@ -25,7 +25,8 @@ STATUS = {0: "MOBA_OK", 1: "MOBA_ERR_INVALID_ARG", 2: "MOBA_ERR_UNSUPPORTED",
 EXPORTS = ("moba_kbar_elems", "moba_workspace_size", "moba_pool_keys", "moba_gate_topk",
            "moba_attn_fwd", "moba_fwd", "moba_route", "moba_attn_past", "moba_attn_self_merge",
            "moba_launches_per_forward", "moba_read_device_error", "moba_status_string",
-           "moba_last_error", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait")
+           "moba_last_error", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait",
+           "moba_host_staging_size", "moba_fwd_host")
 
 
 class MobaError(RuntimeError):
@@ -73,6 +74,10 @@ def load():
         lib.moba_attn_self_merge.argtypes = [P, vp, vp, vp, vp, vp, sz, vp, vp, vp]
         lib.moba_gate_topk_noalloc.argtypes = [P, vp, vp, vp, vp]
         lib.moba_gate_topk_noalloc.restype = ctypes.c_int
+        lib.moba_host_staging_size.argtypes = [P, ctypes.c_int]
+        lib.moba_host_staging_size.restype = sz
+        lib.moba_fwd_host.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
+        lib.moba_fwd_host.restype = ctypes.c_int
         lib.moba_launches_per_forward.argtypes = [P]
         lib.moba_launches_per_forward.restype = ctypes.c_int
         for f in ("moba_pool_keys", "moba_gate_topk", "moba_attn_fwd", "moba_fwd", "moba_route",
@@ -202,6 +207,18 @@ def moba_attn_self_merge(p: MobaParams, Q, K, V, sel, workspace, O, LSE, stream=
 def moba_gate_topk_noalloc(p: MobaParams, Q, Kbar, sel, stream=None) -> None:
     """moba_gate_topk for callers without an allocator: scratch is a fixed array in the library."""
     _check(load().moba_gate_topk_noalloc(p.ref(), _ptr(Q), _ptr(Kbar), _ptr(sel), _stream(stream)))
+
+
+def moba_host_staging_size(p: MobaParams, nstreams: int) -> int:
+    return int(load().moba_host_staging_size(p.ref(), nstreams))
+
+
+def moba_fwd_host(p: MobaParams, Q, K, V, O, LSE, staging, streams) -> None:
+    """Forward on pinned HOST tensors (Q, K, V in; O, LSE out), copies overlapped with the
+    kernels over the given CUDA streams; asynchronous (synchronise the streams afterwards)."""
+    arr = (ctypes.c_void_p * len(streams))(*[_stream(s) for s in streams])
+    _check(load().moba_fwd_host(p.ref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), _ptr(staging),
+                                staging.numel() * staging.element_size(), arr, len(streams)))
 
 
 def moba_launches_per_forward(p: MobaParams) -> int:

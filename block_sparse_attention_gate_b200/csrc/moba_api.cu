@@ -347,6 +347,107 @@ moba_status moba_fwd(const moba_params* p, const void* Q, const void* K, const v
   return attn_stages(g, Q, K, V, sl, w, O, LSE, st, 7);
 }
 
+// ------------------------------------------------------------------ host-buffer forward
+namespace {
+
+// Parameters of one KV-head group as a problem of its own (G query heads, one KV head).
+moba_params group_params(const moba_params* p) {
+  moba_params q = *p;
+  q.num_q_heads = p->num_q_heads / p->num_kv_heads;
+  q.num_kv_heads = 1;
+  return q;
+}
+
+struct HostSlot {
+  char* Q;
+  char* K;
+  char* V;
+  char* O;
+  float* LSE;
+  char* ws;
+  size_t ws_bytes;
+  size_t bytes;
+};
+
+// Device staging of one slot: Q, K, V, O, LSE of one group plus that group's workspace.
+HostSlot carve_slot(const moba::Geom& gg, size_t ws_bytes, char* base) {
+  HostSlot h;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* ptr = base ? base + off : nullptr;
+    off += align256(bytes);
+    return ptr;
+  };
+  const size_t T = (size_t)gg.T, D = (size_t)gg.D, G = (size_t)gg.Hq;
+  h.Q = take(T * G * D * 2);
+  h.K = take(T * D * 2);
+  h.V = take(T * D * 2);
+  h.O = take(T * G * D * 2);
+  h.LSE = (float*)take(T * G * 4);
+  h.ws = take(ws_bytes);
+  h.ws_bytes = ws_bytes;
+  h.bytes = off;
+  return h;
+}
+
+}  // namespace
+
+size_t moba_host_staging_size(const moba_params* p, int nslots) {
+  moba::Geom g;
+  if (make_geom(p, &g) != MOBA_OK || nslots < 1) return 0;
+  moba_params q = group_params(p);
+  moba::Geom gg;
+  if (make_geom(&q, &gg) != MOBA_OK) return 0;
+  const size_t ws = carve(gg, nullptr, nullptr);
+  return (size_t)nslots * carve_slot(gg, ws, nullptr).bytes;
+}
+
+moba_status moba_fwd_host(const moba_params* p, const void* Q, const void* K, const void* V, void* O, float* LSE,
+                          void* staging, size_t staging_bytes, void* const* streams, int nstreams) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0) return MOBA_OK;
+  if (!Q || !K || !V || !O || !LSE) return fail(MOBA_ERR_INVALID_ARG, "a host buffer is NULL");
+  if (!streams || nstreams < 1) return fail(MOBA_ERR_INVALID_ARG, "need at least one stream");
+  const size_t need = moba_host_staging_size(p, nstreams);
+  if (!staging || (((uintptr_t)staging) & 255)) return fail(MOBA_ERR_WORKSPACE, "staging missing or not 256-byte aligned");
+  if (staging_bytes < need) return fail(MOBA_ERR_WORKSPACE, "staging has %zu bytes, %zu needed", staging_bytes, need);
+  moba_params q = group_params(p);
+  moba::Geom gg;
+  MOBA_TRY(make_geom(&q, &gg));
+  MOBA_TRY(check_device(&gg));
+  const size_t ws = carve(gg, nullptr, nullptr);
+  const size_t slot_bytes = carve_slot(gg, ws, nullptr).bytes;
+  const size_t T = (size_t)g.T, D = (size_t)g.D, G = (size_t)gg.Hq;
+  const size_t Hq = (size_t)g.Hq, Hkv = (size_t)g.Hkv;
+  for (int grp = 0; grp < g.Hkv; ++grp) {
+    const int slot = grp % nstreams;
+    cudaStream_t st = (cudaStream_t)streams[slot];
+    HostSlot h = carve_slot(gg, ws, (char*)staging + (size_t)slot * slot_bytes);
+    const char* qh = (const char*)Q + (size_t)grp * G * D * 2;
+    const char* kh = (const char*)K + (size_t)grp * D * 2;
+    const char* vh = (const char*)V + (size_t)grp * D * 2;
+    cudaError_t e = cudaMemcpy2DAsync(h.Q, G * D * 2, qh, Hq * D * 2, G * D * 2, T, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpy2DAsync(h.K, D * 2, kh, Hkv * D * 2, D * 2, T, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpy2DAsync(h.V, D * 2, vh, Hkv * D * 2, D * 2, T, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    moba::Work w;
+    carve(gg, h.ws, &w);
+    e = moba::launch_pool(gg, (const __nv_bfloat16*)h.K, w.kbar, st);
+    if (e != cudaSuccess) return cuda_fail(e, "pool launch");
+    e = moba::launch_gate(gg, (const __nv_bfloat16*)h.Q, w.kbar, w.sel, w, st);
+    if (e != cudaSuccess) return cuda_fail(e, "gate launch");
+    MOBA_TRY(attn_stages(gg, h.Q, h.K, h.V, w.sel, w, h.O, h.LSE, st, 7));
+    char* oh = (char*)O + (size_t)grp * G * D * 2;
+    float* lh = LSE + (size_t)grp * G;
+    e = cudaMemcpy2DAsync(oh, Hq * D * 2, h.O, G * D * 2, G * D * 2, T, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaMemcpy2DAsync(lh, Hq * 4, h.LSE, G * 4, G * 4, T, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  }
+  return MOBA_OK;
+}
+
 const char* moba_status_string(int status) {
   switch (status) {
     case MOBA_OK: return "ok";

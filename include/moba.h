@@ -170,6 +170,26 @@ MOBA_API moba_status moba_attn_self_merge(const moba_params* p, const void* Q, c
 MOBA_API moba_status moba_gate_topk_noalloc(const moba_params* p, const void* Q, const float* Kbar,
                                             int32_t* sel, void* stream);
 
+/*
+ * The whole forward pass on HOST buffers, with the host<->device copies overlapped with the
+ * kernels.  MoBA is independent per KV-head group (each group's queries gate on, and attend
+ * to, that group's keys only), so the problem is cut into its Hkv groups: for each group the
+ * Q/K/V head slices are copied (2D copies, no host repacking) into a device staging slot,
+ * the forward runs on them, and the O/LSE slices are copied back into place.  Group g uses
+ * slot g % nstreams and streams[g % nstreams], so copies of one group overlap the kernels
+ * and copies of others.  Results equal moba_fwd's.
+ *   Q [T, Hq, D], K, V [T, Hkv, D] bf16, O [T, Hq, D] bf16, LSE [T, Hq] fp32: HOST pointers,
+ *     page-locked (pinned) for the copies to be asynchronous and to overlap.
+ *   staging: DEVICE buffer of moba_host_staging_size(p, nstreams) bytes, 256-byte aligned.
+ *   streams: nstreams cudaStream_t handles owned by the caller.
+ * Asynchronous: returns once everything is enqueued; synchronise every stream before
+ * reading O/LSE or reusing the inputs.  cu_seqlens (host and device) as for moba_fwd.
+ */
+MOBA_API size_t moba_host_staging_size(const moba_params* p, int nstreams);
+MOBA_API moba_status moba_fwd_host(const moba_params* p, const void* Q, const void* K, const void* V, void* O,
+                                   float* LSE, void* staging, size_t staging_bytes, void* const* streams,
+                                   int nstreams);
+
 /* Kernel launches one moba_fwd enqueues for these params (host only; -1 if invalid). */
 MOBA_API int moba_launches_per_forward(const moba_params* p);
 
