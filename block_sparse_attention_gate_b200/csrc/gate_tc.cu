@@ -43,9 +43,9 @@ __device__ __forceinline__ bool ranks_before(float sa, int32_t ba, float sb, int
   return sa > sb || (sa == sb && ba < bb);
 }
 
-// kMaxM: compile-time capacity of the running top list (>= top_k - 1), so the list lives
-// in registers and an insertion costs kMaxM compare-and-swap steps.
-template <int D, int kMaxM>
+// kMaxM: compile-time capacity of the running top lists (>= top_k - 1), so the lists live
+// in registers; kLists of them take interleaved candidates to shorten the dependency chain.
+template <int D, int kMaxM, int kLists = (kMaxM <= 4 ? 4 : (kMaxM <= 8 ? 2 : 1))>
 __global__ void __launch_bounds__(kThreads, 2)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmHi,
                    const __grid_constant__ CUtensorMap tmLo, Geom g, int32_t* __restrict__ sel) {
@@ -100,56 +100,101 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ========================================================= epilogue: running top-m
     const int r = tid;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    // Sorted list (best first) of kMaxM slots; the first kMaxM - m slots hold sentinels that
-    // rank before every score and are never displaced, so the m live slots are the last m
-    // and the current m-th best is always the last slot (no runtime indexing).
-    float ts_[kMaxM];
-    int32_t tb_[kMaxM];
+    // kLists independent sorted lists (best first) of kMaxM slots each; candidate column x
+    // of a 32-column group goes to list x % kLists, so kLists insertion chains run side by
+    // side.  In each list the first kMaxM - m slots hold sentinels that rank before every
+    // score and are never displaced, so the m live slots are the last m and the current
+    // m-th best is always the last slot (no runtime indexing).
+    float ts_[kLists][kMaxM];
+    int32_t tb_[kLists][kMaxM];
 #pragma unroll
-    for (int q = 0; q < kMaxM; ++q) {
-      const bool live = q >= kMaxM - m;
-      ts_[q] = live ? -FLT_MAX : FLT_MAX;
-      tb_[q] = live ? INT32_MAX : -1;
-    }
+    for (int j = 0; j < kLists; ++j)
+#pragma unroll
+      for (int q = 0; q < kMaxM; ++q) {
+        const bool live = q >= kMaxM - m;
+        ts_[j][q] = live ? -FLT_MAX : FLT_MAX;
+        tb_[j][q] = live ? INT32_MAX : -1;
+      }
+    // Candidates reach a list in ascending block index, so a new one ranks after every
+    // listed entry whose score is >= its own (ties go to the lower index) and before the
+    // rest: the list shifts down by one from that position.  A score at or below the last
+    // slot leaves the list unchanged, so the update needs no branch.
+    auto insert = [&](float (&ls)[kMaxM], int32_t (&lb)[kMaxM], float sc, int32_t b) {
+      bool ge[kMaxM];
+#pragma unroll
+      for (int q = 0; q < kMaxM; ++q) ge[q] = ls[q] >= sc;
+#pragma unroll
+      for (int q = kMaxM - 1; q >= 1; --q) {
+        ls[q] = ge[q] ? ls[q] : (ge[q - 1] ? sc : ls[q - 1]);
+        lb[q] = ge[q] ? lb[q] : (ge[q - 1] ? b : lb[q - 1]);
+      }
+      ls[0] = ge[0] ? ls[0] : sc;
+      lb[0] = ge[0] ? lb[0] : b;
+    };
+    // One 32-column group of S; columns at or past the query block i score -FLT_MAX, which
+    // never enters a list.
+    auto scan = [&](const uint32_t (&v)[32], int32_t b0) {
+#pragma unroll
+      for (int x = 0; x < 32; ++x) {
+        const int32_t b = b0 + x;
+        const float sc = b < i ? __uint_as_float(v[x]) : -FLT_MAX;
+        if constexpr (kMaxM <= 4) {
+          insert(ts_[x % kLists], tb_[x % kLists], sc, b);
+        } else {
+          if (sc > ts_[x % kLists][kMaxM - 1]) insert(ts_[x % kLists], tb_[x % kLists], sc, b);
+        }
+      }
+    };
     for (int c = 0; c < nch && ok; ++c) {
       const int buf = c & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[kTFull0 + buf], (c >> 1) & 1, g.err));
       if (!ok) break;
       tc_fence_after();
       const int c0 = c * kCand;
-      const int ncand = min(kCand, i - c0);
-      for (int x0 = 0; x0 < ncand; x0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + buf * kCand + x0, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int32_t b = c0 + x0 + x;
-          float sc = __uint_as_float(v[x]);
-          if (b < i && ranks_before(sc, b, ts_[kMaxM - 1], tb_[kMaxM - 1])) {
-            int32_t cb = b;
-#pragma unroll
-            for (int q = 0; q < kMaxM; ++q) {
-              const bool take = ranks_before(sc, cb, ts_[q], tb_[q]);
-              const float os = ts_[q];
-              const int32_t ob = tb_[q];
-              ts_[q] = take ? sc : os;
-              tb_[q] = take ? cb : ob;
-              sc = take ? os : sc;
-              cb = take ? ob : cb;
-            }
-          }
+      const int ngrp = (min(kCand, i - c0) + 31) / 32;
+      const uint32_t t0 = tmem + lane_off + buf * kCand;
+      // The next group's TMEM load is in flight while the current group is scanned.
+      uint32_t va[32], vb[32];
+      tmem_ld32(t0, va);
+      tmem_wait_ld(va);
+      for (int gi = 0; gi < ngrp; gi += 2) {
+        if (gi + 1 < ngrp) tmem_ld32(t0 + (gi + 1) * 32, vb);
+        scan(va, c0 + gi * 32);
+        if (gi + 1 < ngrp) {
+          tmem_wait_ld(vb);
+          if (gi + 2 < ngrp) tmem_ld32(t0 + (gi + 2) * 32, va);
+          scan(vb, c0 + (gi + 1) * 32);
+          if (gi + 2 < ngrp) tmem_wait_ld(va);
         }
       }
       tc_fence_before();
       mbar_arrive(&bars[kTFree0 + buf]);
     }
+    // Fold lists 1.. into list 0 (entries are no longer in index order: full comparison).
+#pragma unroll
+    for (int j = 1; j < kLists; ++j)
+#pragma unroll
+      for (int p = 0; p < kMaxM; ++p) {
+        if (p < kMaxM - m) continue;
+        float sc = ts_[j][p];
+        int32_t cb = tb_[j][p];
+#pragma unroll
+        for (int q = 0; q < kMaxM; ++q) {
+          const bool take = ranks_before(sc, cb, ts_[0][q], tb_[0][q]);
+          const float os = ts_[0][q];
+          const int32_t ob = tb_[0][q];
+          ts_[0][q] = take ? sc : os;
+          tb_[0][q] = take ? cb : ob;
+          sc = take ? os : sc;
+          cb = take ? ob : cb;
+        }
+      }
     if (ok && r < nrows) {
       int32_t* out = sel + ((int64_t)(q0 + r) * g.Hq + h) * g.k;
       out[0] = i;
 #pragma unroll
       for (int q = 0; q < kMaxM; ++q)
-        if (q >= kMaxM - m) out[1 + q - (kMaxM - m)] = tb_[q];
+        if (q >= kMaxM - m) out[1 + q - (kMaxM - m)] = tb_[0][q];
       for (int q = 1 + m; q < g.k; ++q) out[q] = -1;
     }
   } else if (lane == 0) {
