@@ -13,11 +13,15 @@
 // online softmax; zhuoshang.net, "MoBA是什么？…", section "MoBA的技术原理": causal mask inside
 // the current block.)
 //
-// Per 128-key chunk j:  S_j = Q K_j^T  (tcgen05, fp32 in TMEM, double-buffered)
-//                       softmax rows in registers (one thread per row), P_j -> smem (bf16)
-//                       O += P_j V_j    (tcgen05, fp32 accumulator in TMEM)
-// Warp roles: warps 0-3 softmax + epilogue (thread r owns row r = TMEM lane r), warp 4 TMA
-// producer (K/V chunks, two stages), warp 5 TMEM owner + MMA issuer.
+// Two 128-row query tiles per CTA.  Per 128-key chunk j of tile t:
+//   S_t = Q_t K_j^T   (tcgen05 SS MMA, fp32 in TMEM)
+//   softmax of S_t in registers (one thread per row = TMEM lane), P_t (bf16) written back
+//   over the first half of S_t's TMEM columns
+//   O_t += P_t V_j    (tcgen05 TS MMA, A read from TMEM, fp32 accumulator in TMEM)
+// The tensor core works on one tile while the other tile's softmax runs.
+// Warp roles: warps 0-3 softmax + epilogue of tile 0, warps 4-7 of tile 1, warp 8 TMA
+// producer (K/V chunks, two stages), warp 9 TMEM owner + MMA issuer (the whole warp runs the
+// issue loop; one elected lane issues each tcgen05.mma), warps 10-11 idle (register donors).
 #include <cudaTypedefs.h>
 #include <float.h>
 
@@ -205,12 +209,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
       }
     }
+    // own mode: this row's past partials exist before this kernel starts (the past-block
+    // attention ran earlier), so their ids and LSEs are read here, while the Q gather is in
+    // flight, and their O rows are pulled into L2 for the merge at the end.
+    int32_t pe[kMaxTopK];
+    float pw[kMaxTopK];
+    int np = 0;
     {  // gather this row of Q into tile t (zeros for padding rows)
       const __nv_bfloat16* src = qrow >= 0 ? a.Q + qrow * D : a.Q;
       const uint32_t nb = qrow >= 0 ? 16u : 0u;
       const uint32_t sQ = smem_u32(smem + L::kQ + t * L::kTile);
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) cp_async_16(sQ + sw128_offset(r, c, kRows), src + c * 8, nb);
+      if constexpr (kOwn) {
+        if (r < T_.nrows) {
+          int32_t bsel[kMaxTopK - 1];
+#pragma unroll
+          for (int q = 0; q < kMaxTopK - 1; ++q) bsel[q] = q + 1 < g.k ? __ldg(a.sel + qrow * g.k + q + 1) : -1;
+#pragma unroll
+          for (int q = 0; q < kMaxTopK - 1; ++q)
+            if (bsel[q] >= 0 && bsel[q] < i_blk) pe[np++] = (int32_t)(qrow * (g.k - 1) + q);
+#pragma unroll
+          for (int q = 0; q < kMaxTopK - 1; ++q)
+            if (q < np) {
+              pw[q] = __ldg(a.part_lse + pe[q]);
+              const float* po = a.part_o + (int64_t)pe[q] * D;
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) prefetch_l2(po + c * 32);
+            }
+        }
+      }
       cp_async_wait_all();
       fence_proxy_async_smem();
       mbar_arrive(&bars[kQFull]);
@@ -308,11 +336,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const float lse_row = (m + __log2f(l)) * kLn2;
-      // Each warp stages its 32 rows (fp32, D columns) in shared memory that no MMA reads any
-      // more (this tile's Q buffer and one K stage: every QK^T MMA completed before the O
-      // barrier fired), then writes whole rows with coalesced stores.  16-byte chunks of a
-      // staged row are XOR-swizzled by (row mod 8) to spread the row-per-thread writes over
-      // the banks.
+      // own mode: each warp stages its 32 rows (fp32, D columns) in shared memory that no MMA
+      // reads any more (this tile's Q buffer and one K stage: every QK^T MMA completed before
+      // the O barrier fired), then merges and writes whole rows cooperatively.  16-byte chunks
+      // of a staged row are XOR-swizzled by (row mod 8) to spread the row-per-thread writes
+      // over the banks.
       const int wq = warp & 3;
       float* stg = reinterpret_cast<float*>(smem + (wq < 2 ? L::kQ : L::kK0) + t * L::kTile + (wq & 1) * (L::kTile / 2));
       auto stg_at = [&](int row, int col) -> float* {
@@ -321,21 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float scale_row = inv_l;
       // own mode: merge weights of this row (own block and its past partials)
       float M = lse_row, inv_w = 1.f;
-      int32_t pe[kMaxTopK];
-      float pw[kMaxTopK];
-      int np = 0;
       if constexpr (kOwn) {
-        if (r < T_.nrows) {
-          for (int slot = 1; slot < g.k; ++slot) {
-            const int32_t b = __ldg(a.sel + qrow * g.k + slot);
-            if (b >= 0 && b < i_blk) {
-              pe[np] = (int32_t)(qrow * (g.k - 1) + slot - 1);
-              pw[np] = __ldg(a.part_lse + pe[np]);
-              M = fmaxf(M, pw[np]);
-              ++np;
-            }
-          }
-        }
+        for (int q = 0; q < np; ++q) M = fmaxf(M, pw[q]);
         const float w_self = __expf(lse_row - M);
         float sumw = w_self;
         for (int q = 0; q < np; ++q) {
@@ -349,27 +364,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         if (r < T_.nrows) a.part_lse[e] = lse_row;
       }
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int x = 0; x < 32; x += 4)
-          *reinterpret_cast<float4*>(stg_at(lane, c * 32 + x)) =
-              make_float4(__uint_as_float(o[x]) * scale_row, __uint_as_float(o[x + 1]) * scale_row,
-                          __uint_as_float(o[x + 2]) * scale_row, __uint_as_float(o[x + 3]) * scale_row);
-      }
-      __syncwarp();
       if constexpr (!kOwn) {
-        for (int rr = 0; rr < 32; ++rr) {
-          const int32_t er = __shfl_sync(0xffffffffu, e, rr);
-          if (er < 0) continue;
-          float* dst = a.part_o + (int64_t)er * D + lane;
+        // Each thread stages its own row (fp32; rows padded by 16 bytes so the row-per-thread
+        // 16-byte writes spread over the banks) and hands it to the TMA engine as one bulk
+        // copy to the row's partial slot.  The copies drain to memory on their own; the thread
+        // only waits until the engine has read the staged row.  Tile 0's warps stage in the Q
+        // and K buffers (free: the O barrier implies every QK^T MMA completed); tile 1's
+        // warps, whose O barrier follows the last MMA of the CTA, continue into the V buffers.
+        constexpr int kStgRow = D + 4;
+        static_assert(8 * 32 * kStgRow * 4 <= L::kBar && 4 * 32 * kStgRow * 4 <= L::kV0, "staging rows");
+        float* srow = reinterpret_cast<float*>(smem + L::kQ) + (warp * 32 + lane) * kStgRow;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) dst[c * 32] = *stg_at(rr, c * 32 + lane);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; x += 4)
+            *reinterpret_cast<float4*>(srow + c * 32 + x) =
+                make_float4(__uint_as_float(o[x]) * scale_row, __uint_as_float(o[x + 1]) * scale_row,
+                            __uint_as_float(o[x + 2]) * scale_row, __uint_as_float(o[x + 3]) * scale_row);
+        }
+        if (e >= 0) {
+          fence_proxy_async_smem();
+          bulk_store_s2g(a.part_o + (int64_t)e * D, smem_u32(srow), D * 4);
+          bulk_commit();
+          bulk_wait_read_all();
         }
       } else {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; x += 4)
+            *reinterpret_cast<float4*>(stg_at(lane, c * 32 + x)) =
+                make_float4(__uint_as_float(o[x]) * scale_row, __uint_as_float(o[x + 1]) * scale_row,
+                            __uint_as_float(o[x + 2]) * scale_row, __uint_as_float(o[x + 3]) * scale_row);
+        }
+        __syncwarp();
         // eight rows at a time, so their partial rows are all in flight together
         constexpr int kU = 8;
         for (int rr0 = 0; rr0 < 32; rr0 += kU) {
@@ -435,64 +469,63 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 9) {
-    // ========================================================= MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(kRows, kBN, false, false);
-      constexpr uint32_t idO = idesc_bf16(kRows, D, false, true);
-      const uint32_t sQ = smem_u32(smem + L::kQ);
-      const uint32_t sK0 = smem_u32(smem + L::kK0);
-      const uint32_t sV0 = smem_u32(smem + L::kV0);
-      auto issue_s = [&](int t, int j) {
-        const uint32_t qb = sQ + t * L::kTile, kb = sK0 + (j & 1) * L::kTile;
+    // ========================================================= MMA issuer (whole warp, one elected lane issues)
+    constexpr uint32_t idS = idesc_bf16(kRows, kBN, false, false);
+    constexpr uint32_t idO = idesc_bf16(kRows, D, false, true);
+    const uint32_t sQ = smem_u32(smem + L::kQ);
+    const uint32_t sK0 = smem_u32(smem + L::kK0);
+    const uint32_t sV0 = smem_u32(smem + L::kV0);
+    auto issue_s = [&](int t, int j) {
+      const uint32_t qb = sQ + t * L::kTile, kb = sK0 + (j & 1) * L::kTile;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
-          mma_bf16_ss(tmem + kColS + t * kBN, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idS,
-                      kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars[kSFull0 + t]);
-      };
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t vb = sV0 + (j & 1) * L::kTile;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+        mma_bf16_ss_warp(tmem + kColS + t * kBN, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                         idS, kk > 0 ? 1u : 0u);
+      }
+      mma_commit_warp(&bars[kSFull0 + t]);
+    };
+    auto issue_pv = [&](int t, int j) {
+      const uint32_t vb = sV0 + (j & 1) * L::kTile;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_bf16_ts(tmem + kColO + t * 128, tmem + kColS + t * kBN + kColP + kk * 8,
-                      sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
-      };
-      ok = mbar_wait(&bars[kQFull], 0, g.err) && mbar_wait(&bars[kKFull0], 0, g.err);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        mma_commit(&bars[kKEmpty0]);
-      }
-      for (int j = 0; j < nchunks && ok; ++j) {
-        const bool more = j + 1 < nchunks;
-        ok = mbar_wait(&bars[kVFull0 + (j & 1)], (j >> 1) & 1, g.err) && mbar_wait(&bars[kPFull0], j & 1, g.err);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(0, j);
-        if (!more) mma_commit(&bars[kOFull0]);
-        if (more) {
-          ok = mbar_wait(&bars[kKFull0 + ((j + 1) & 1)], ((j + 1) >> 1) & 1, g.err);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(0, j + 1);
-        }
-        ok = mbar_wait(&bars[kPFull1], j & 1, g.err);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, j);
-        mma_commit(&bars[kVEmpty0 + (j & 1)]);
-        if (!more) mma_commit(&bars[kOFull1]);
-        if (more) {
-          issue_s(1, j + 1);
-          mma_commit(&bars[kKEmpty0 + ((j + 1) & 1)]);
-        }
-      }
-      mma_commit(&bars[kDone]);
-      mbar_wait(&bars[kDone], 0, g.err);
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        mma_bf16_ts_warp(tmem + kColO + t * 128, tmem + kColS + t * kBN + kColP + kk * 8,
+                         sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
+    };
+    ok = mbar_wait_warp(&bars[kQFull], 0, g.err) && mbar_wait_warp(&bars[kKFull0], 0, g.err);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0, 0);
+      issue_s(1, 0);
+      mma_commit_warp(&bars[kKEmpty0]);
     }
+    for (int j = 0; j < nchunks && ok; ++j) {
+      const bool more = j + 1 < nchunks;
+      ok = mbar_wait_warp(&bars[kVFull0 + (j & 1)], (j >> 1) & 1, g.err) &&
+           mbar_wait_warp(&bars[kPFull0], j & 1, g.err);
+      if (!ok) break;
+      tc_fence_after();
+      issue_pv(0, j);
+      if (!more) mma_commit_warp(&bars[kOFull0]);
+      if (more) {
+        ok = mbar_wait_warp(&bars[kKFull0 + ((j + 1) & 1)], ((j + 1) >> 1) & 1, g.err);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(0, j + 1);
+      }
+      ok = mbar_wait_warp(&bars[kPFull1], j & 1, g.err);
+      if (!ok) break;
+      tc_fence_after();
+      issue_pv(1, j);
+      mma_commit_warp(&bars[kVEmpty0 + (j & 1)]);
+      if (!more) mma_commit_warp(&bars[kOFull1]);
+      if (more) {
+        issue_s(1, j + 1);
+        mma_commit_warp(&bars[kKEmpty0 + ((j + 1) & 1)]);
+      }
+    }
+    mma_commit_warp(&bars[kDone]);
+    mbar_wait_warp(&bars[kDone], 0, g.err);
   }
 
   // ------------------------------------------------------------- teardown

@@ -22,7 +22,7 @@ namespace moba {
 
 namespace {
 
-constexpr int kThreads = 160;     // warps 0-3 epilogue, warp 4 TMA + MMA
+constexpr int kThreads = 160;     // warps 0-3 epilogue, warp 4 TMA + MMA (whole warp)
 constexpr int kRows = 128;        // query rows per CTA
 constexpr int kCand = 128;        // candidate blocks per chunk
 constexpr int kBoxRows = 64;      // candidate rows per TMA box
@@ -197,9 +197,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (q >= kMaxM - m) out[1 + q - (kMaxM - m)] = tb_[0][q];
       for (int q = 1 + m; q < g.k; ++q) out[q] = -1;
     }
-  } else if (lane == 0) {
-    // ========================================================= TMA + MMA issuer
+  } else {
+    // ========================================================= TMA + MMA issuer (warp 4)
+    // The whole warp runs this loop: lane 0 issues the TMA copies, one elected lane the MMAs.
     auto load_chunk = [&](int c, bool with_q) {
+      if (lane != 0) return;
       const int c0 = c * kCand;
       const int ncand = min(kCand, i - c0);
       const int nbox = (ncand + kBoxRows - 1) / kBoxRows;
@@ -217,17 +219,20 @@ __global__ void __launch_bounds__(kThreads, 2)
           tma_load_3d(smem + L::kLo + off, &tmLo, &bars[kFull], hh * 64, gk, row);
         }
     };
-    prefetch_tmap(&tmQ);
-    prefetch_tmap(&tmHi);
-    prefetch_tmap(&tmLo);
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmHi);
+      prefetch_tmap(&tmLo);
+    }
     load_chunk(0, true);
+    __syncwarp();
     const uint32_t sQ = smem_u32(smem + L::kQ);
     const uint32_t sHi = smem_u32(smem + L::kHi);
     const uint32_t sLo = smem_u32(smem + L::kLo);
     for (int c = 0; c < nch && ok; ++c) {
       const int buf = c & 1;
-      ok = mbar_wait(&bars[kFull], c & 1, g.err);
-      if (ok && c >= 2) ok = mbar_wait(&bars[kTFree0 + buf], ((c >> 1) - 1) & 1, g.err);
+      ok = mbar_wait_warp(&bars[kFull], c & 1, g.err);
+      if (ok && c >= 2) ok = mbar_wait_warp(&bars[kTFree0 + buf], ((c >> 1) - 1) & 1, g.err);
       if (!ok) break;
       tc_fence_after();
       const int ncand = min(kCand, i - c * kCand);
@@ -238,19 +243,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t koff = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
         const uint32_t boff = (kk >> 2) * (kCand * 128) + (kk & 3) * 32;
         const uint64_t ad = sdesc_sw128(sQ + koff, 16, 1024);
-        mma_bf16_ss(tmem + buf * kCand, ad, sdesc_sw128(sHi + boff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-        mma_bf16_ss(tmem + buf * kCand, ad, sdesc_sw128(sLo + boff, 16, 1024), idesc, 1u);
+        mma_bf16_ss_warp(tmem + buf * kCand, ad, sdesc_sw128(sHi + boff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        mma_bf16_ss_warp(tmem + buf * kCand, ad, sdesc_sw128(sLo + boff, 16, 1024), idesc, 1u);
       }
-      mma_commit(&bars[kTFull0 + buf]);
+      mma_commit_warp(&bars[kTFull0 + buf]);
       if (c + 1 < nch) {
-        mma_commit(&bars[kKFree]);
-        ok = mbar_wait(&bars[kKFree], c & 1, g.err);
+        mma_commit_warp(&bars[kKFree]);
+        ok = mbar_wait_warp(&bars[kKFree], c & 1, g.err);
         if (!ok) break;
         load_chunk(c + 1, false);
+        __syncwarp();
       }
     }
-    mma_commit(&bars[kGDone]);
-    mbar_wait(&bars[kGDone], 0, g.err);
+    mma_commit_warp(&bars[kGDone]);
+    mbar_wait_warp(&bars[kGDone], 0, g.err);
   }
   __syncthreads();
   if (warp == 4) {
