@@ -21,7 +21,8 @@
 // The tensor core works on one tile while the other tile's softmax runs.
 // Warp roles: warps 0-3 softmax + epilogue of tile 0, warps 4-7 of tile 1, warp 8 TMA
 // producer (K/V chunks, two stages), warp 9 TMEM owner + MMA issuer (the whole warp runs the
-// issue loop; one elected lane issues each tcgen05.mma), warps 10-11 idle (register donors).
+// issue loop; one elected lane issues each tcgen05.mma), warps 10-11 register donors (in own
+// mode they also prefetch the merge inputs into L2).
 #include <cudaTypedefs.h>
 #include <float.h>
 
@@ -209,36 +210,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
       }
     }
-    // own mode: this row's past partials exist before this kernel starts (the past-block
-    // attention ran earlier), so their ids and LSEs are read here, while the Q gather is in
-    // flight, and their O rows are pulled into L2 for the merge at the end.
-    int32_t pe[kMaxTopK];
-    float pw[kMaxTopK];
-    int np = 0;
     {  // gather this row of Q into tile t (zeros for padding rows)
       const __nv_bfloat16* src = qrow >= 0 ? a.Q + qrow * D : a.Q;
       const uint32_t nb = qrow >= 0 ? 16u : 0u;
       const uint32_t sQ = smem_u32(smem + L::kQ + t * L::kTile);
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) cp_async_16(sQ + sw128_offset(r, c, kRows), src + c * 8, nb);
-      if constexpr (kOwn) {
-        if (r < T_.nrows) {
-          int32_t bsel[kMaxTopK - 1];
-#pragma unroll
-          for (int q = 0; q < kMaxTopK - 1; ++q) bsel[q] = q + 1 < g.k ? __ldg(a.sel + qrow * g.k + q + 1) : -1;
-#pragma unroll
-          for (int q = 0; q < kMaxTopK - 1; ++q)
-            if (bsel[q] >= 0 && bsel[q] < i_blk) pe[np++] = (int32_t)(qrow * (g.k - 1) + q);
-#pragma unroll
-          for (int q = 0; q < kMaxTopK - 1; ++q)
-            if (q < np) {
-              pw[q] = __ldg(a.part_lse + pe[q]);
-              const float* po = a.part_o + (int64_t)pe[q] * D;
-#pragma unroll
-              for (int c = 0; c < D / 32; ++c) prefetch_l2(po + c * 32);
-            }
-        }
-      }
       cp_async_wait_all();
       fence_proxy_async_smem();
       mbar_arrive(&bars[kQFull]);
@@ -347,9 +324,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         return stg + row * D + ((((col >> 2) ^ (row & 7)) << 2) | (col & 3));
       };
       float scale_row = inv_l;
-      // own mode: merge weights of this row (own block and its past partials)
+      // own mode: merge weights of this row (own block and its past partials).  The loads
+      // are independent of one another (all slots, then all LSEs) and hit L2: warps 10-11
+      // pulled these lines in while the block attention ran.
       float M = lse_row, inv_w = 1.f;
+      int32_t pe[kMaxTopK];
+      float pw[kMaxTopK];
+      int np = 0;
       if constexpr (kOwn) {
+        if (r < T_.nrows) {
+          int32_t bsel[kMaxTopK - 1];
+#pragma unroll
+          for (int q = 0; q < kMaxTopK - 1; ++q) bsel[q] = q + 1 < g.k ? __ldg(a.sel + qrow * g.k + q + 1) : -1;
+#pragma unroll
+          for (int q = 0; q < kMaxTopK - 1; ++q)
+            if (bsel[q] >= 0 && bsel[q] < i_blk) pe[np++] = (int32_t)(qrow * (g.k - 1) + q);
+#pragma unroll
+          for (int q = 0; q < kMaxTopK - 1; ++q)
+            if (q < np) pw[q] = __ldg(a.part_lse + pe[q]);
+        }
         for (int q = 0; q < np; ++q) M = fmaxf(M, pw[q]);
         const float w_self = __expf(lse_row - M);
         float sumw = w_self;
@@ -444,6 +437,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < D / 32; ++c) dst[c * 32] = __float2bfloat16_rn(acc[u][c]);
           }
         }
+      }
+    }
+  } else if (warp >= 10) {
+    // ========================================================= own mode: merge-input prefetch
+    // Warps 10-11 have no role in the attention itself.  In own mode they pull every row's
+    // merge inputs into L2 while the block attention runs (the past partials exist before
+    // this kernel starts): the chosen-block slots, then each past partial's LSE and O row.
+    if constexpr (kOwn) {
+      for (int rr = tid - 10 * 32; rr < 2 * kRows; rr += 64) {
+        const TileInfo& T_ = ti[rr / kRows];
+        const int r = rr % kRows;
+        if (r >= T_.nrows) continue;
+        const int64_t qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
+        int32_t bsel[kMaxTopK - 1];
+#pragma unroll
+        for (int q = 0; q < kMaxTopK - 1; ++q) bsel[q] = q + 1 < g.k ? __ldg(a.sel + qrow * g.k + q + 1) : -1;
+#pragma unroll
+        for (int q = 0; q < kMaxTopK - 1; ++q)
+          if (bsel[q] >= 0 && bsel[q] < i_blk) {
+            const int64_t pq = qrow * (g.k - 1) + q;
+            prefetch_l2(a.part_lse + pq);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) prefetch_l2(a.part_o + pq * D + c * 32);
+          }
       }
     }
   } else if (warp == 8) {
