@@ -57,6 +57,7 @@ struct AttnArgs {
   const int32_t* sel;
   const int32_t* offsets;
   const int32_t* tile_off;
+  const int32_t* tile_bucket;
   const int32_t* rows;
   float* part_o;
   float* part_lse;
@@ -93,7 +94,8 @@ struct TileInfo {
 
 template <int D, bool kOwn>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -110,11 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t total = __ldg(a.tile_off + g.nbk);
     const int32_t tile = (int32_t)blockIdx.x;
     if (tile >= total) return;
-    int64_t lo = 0, hi = g.nbk - 1;  // last bucket whose first tile is <= tile
-    while (lo < hi) {
-      const int64_t mid = (lo + hi + 1) >> 1;
-      if (__ldg(a.tile_off + mid) <= tile) lo = mid; else hi = mid - 1;
-    }
+    const int64_t lo = __ldg(a.tile_bucket + tile);  // this tile's bucket
     const int32_t b = (int32_t)(lo % g.MB);
     s = (int)((lo / g.MB) % g.num_seqs);
     gk = (int)(lo / ((int64_t)g.MB * g.num_seqs));
@@ -176,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
   }
   if (tid == 0) {
-    mbar_init(&bars[kQFull], 2 * kRows);
+    mbar_init(&bars[kQFull], kOwn ? 1 : 2 * kRows);  // own: one TMA transaction; past: every row's gather
     for (int q = 0; q < 2; ++q) {
       mbar_init(&bars[kKFull0 + q], 1);
       mbar_init(&bars[kKEmpty0 + q], 1);
@@ -210,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
       }
     }
-    {  // gather this row of Q into tile t (zeros for padding rows)
+    if constexpr (!kOwn) {  // gather this row of Q into tile t (zeros for padding rows)
       const __nv_bfloat16* src = qrow >= 0 ? a.Q + qrow * D : a.Q;
       const uint32_t nb = qrow >= 0 ? 16u : 0u;
       const uint32_t sQ = smem_u32(smem + L::kQ + t * L::kTile);
@@ -412,22 +410,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) acc[u][c] = *stg_at(rr0 + u, c * 32 + lane);
           }
-          for (int q = 0; q < npmax; ++q) {
-            float tmp[kU][D / 32];
+          // partials two at a time: the loads of both are in flight together
+          for (int q = 0; q < npmax; q += 2) {
+            float tmp[2][kU][D / 32];
+            float wv[2];
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-              const int32_t pq = __shfl_sync(0xffffffffu, pe[q], rr0 + u);
-              const float* src = a.part_o + (int64_t)pq * D + lane;
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int qq = q + h2;
+              const int32_t pv = qq < np ? pe[qq] : 0;
+              wv[h2] = qq < np ? pw[qq] : 0.f;
 #pragma unroll
-              for (int c = 0; c < D / 32; ++c) tmp[u][c] = q < npr[u] ? __ldg(src + c * 32) : 0.f;
+              for (int u = 0; u < kU; ++u) {
+                const int32_t pq = __shfl_sync(0xffffffffu, pv, rr0 + u);
+                const float* src = a.part_o + (int64_t)pq * D + lane;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) tmp[h2][u][c] = qq < npr[u] ? __ldg(src + c * 32) : 0.f;
+              }
             }
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-              const float wgt = __shfl_sync(0xffffffffu, pw[q], rr0 + u);
-              if (q < npr[u])
+            for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) acc[u][c] = fmaf(wgt, tmp[u][c], acc[u][c]);
-            }
+              for (int u = 0; u < kU; ++u) {
+                const float wgt = __shfl_sync(0xffffffffu, wv[h2], rr0 + u);
+                if (q + h2 < npr[u])
+#pragma unroll
+                  for (int c = 0; c < D / 32; ++c) acc[u][c] = fmaf(wgt, tmp[h2][u][c], acc[u][c]);
+              }
           }
 #pragma unroll
           for (int u = 0; u < kU; ++u) {
@@ -468,6 +476,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      if constexpr (kOwn) {  // both Q tiles: 128 consecutive tokens of one head each
+        prefetch_tmap(&tmQ);
+        mbar_expect_tx(&bars[kQFull], 2 * L::kTile);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int hh = 0; hh < D / 64; ++hh)
+            tma_load_3d(smem + L::kQ + t * L::kTile + hh * kRows * 128, &tmQ, &bars[kQFull], hh * 64, ti[t].h,
+                        ti[t].q0);
+      }
       for (int j = 0; j < nchunks && ok; ++j) {
         const int st = j & 1, u = j >> 1;
         const int tok = key0 + j * kBN;
@@ -557,12 +575,18 @@ template <int D, bool kOwn>
 cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                       const int32_t* sel, const Work& w, __nv_bfloat16* O, float* LSE, dim3 grid, int head_pairs,
                       cudaStream_t st) {
-  CUtensorMap tk, tv;
+  CUtensorMap tq, tk, tv;
   cudaError_t e = make_rows_map(&tk, K, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
+  if (kOwn) {
+    e = make_rows_map(&tq, Q, (uint64_t)g.T, g.Hq, D, kRows);
+    if (e != cudaSuccess) return e;
+  } else {
+    tq = tk;  // unused: past mode gathers its Q rows
+  }
   e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
-  AttnArgs a{g, Q, sel, w.offsets, w.tile_off, w.rows, w.part_o, w.part_lse, O, LSE, head_pairs};
+  AttnArgs a{g, Q, sel, w.offsets, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, O, LSE, head_pairs};
   const int smem = Layout<D>::kAlloc;
   e = cudaFuncSetAttribute(attn_tc_kernel<D, kOwn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -571,7 +595,7 @@ cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16
   e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D, kOwn>);
   if (e != cudaSuccess) return e;
   if ((uint32_t)fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
-  attn_tc_kernel<D, kOwn><<<grid, kThreads, smem, st>>>(tk, tv, a);
+  attn_tc_kernel<D, kOwn><<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 
@@ -580,7 +604,7 @@ cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16
 cudaError_t launch_attn_past(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                              const __nv_bfloat16* V, const Work& w, cudaStream_t st) {
   if (g.T == 0 || g.k < 2 || g.R == 0) return cudaSuccess;
-  const int64_t tiles = (g.R + kPastTileRows - 1) / kPastTileRows + g.nbk;  // bound on routed tile pairs
+  const int64_t tiles = past_tiles(g);  // bound on routed tile pairs
   dim3 grid((unsigned)tiles);
   if (g.D == 64) return launch_tc<64, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, grid, 0, st);
   return launch_tc<128, false>(g, Q, K, V, nullptr, w, nullptr, nullptr, grid, 0, st);

@@ -121,6 +121,7 @@ size_t carve(const moba::Geom& g, char* base, moba::Work* w) {
   x.offsets = (int32_t*)take(sizeof(int32_t) * (size_t)(g.nbk + 1));
   x.cursors = (int32_t*)take(sizeof(int32_t) * (size_t)g.nbk);
   x.tile_off = (int32_t*)take(sizeof(int32_t) * (size_t)(g.nbk + 1));
+  x.tile_bucket = (int32_t*)take(sizeof(int32_t) * (size_t)moba::past_tiles(g));
   x.rows = (int32_t*)take(sizeof(int32_t) * (size_t)g.R);
   x.part_o = (float*)take(sizeof(float) * (size_t)g.R * g.D);
   x.part_lse = (float*)take(sizeof(float) * (size_t)g.R);

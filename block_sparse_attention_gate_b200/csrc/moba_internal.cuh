@@ -29,6 +29,12 @@ struct Geom {
   int* err;           // device error word (bounded waits that gave up), never null
 };
 
+// Upper bound on the past-block attention tiles (kPastTileRows rows each): every bucket's
+// last tile may be partial.
+__host__ __device__ inline int64_t past_tiles(const Geom& g) {
+  return (g.R + kPastTileRows - 1) / kPastTileRows + g.nbk;
+}
+
 __device__ __forceinline__ int32_t seq_start(const Geom& g, int s) {
   return g.cu ? __ldg(g.cu + s) : s * g.L;
 }
@@ -52,6 +58,7 @@ struct Work {
   int32_t* offsets;   // [nbk + 1] exclusive scan of counts
   int32_t* cursors;   // [nbk] scatter cursors
   int32_t* tile_off;  // [nbk + 1] exclusive scan of per-bucket tile counts
+  int32_t* tile_bucket;  // [past_tiles(g)] bucket of each past-attention tile
   int32_t* rows;      // [R] routed partial ids, grouped by bucket
   float* part_o;      // [R, D] normalised partial outputs
   float* part_lse;    // [R] partial log-sum-exp

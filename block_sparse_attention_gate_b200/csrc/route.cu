@@ -18,11 +18,15 @@ __device__ __forceinline__ int64_t bucket_of(const Geom& g, int gk, int s, int32
 }
 
 // grid (MB, num_seqs, Hkv): CTA = query block i of sequence s, KV head g
+// The scatter pass also fills the tile -> bucket table: CTA (i, s, g) writes the tiles of
+// bucket (g, s, i - 1), so every bucket that can hold rows is covered exactly once.
 template <bool kScatter>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geom g, const int32_t* __restrict__ sel,
                                                             int32_t* __restrict__ counts,
                                                             int32_t* __restrict__ cursors,
-                                                            int32_t* __restrict__ rows) {
+                                                            int32_t* __restrict__ rows,
+                                                            const int32_t* __restrict__ tile_off,
+                                                            int32_t* __restrict__ tile_bucket) {
   extern __shared__ int32_t hist[];  // [i] counts, then [i] bases (scatter)
   const int i = blockIdx.x, s = blockIdx.y, gk = blockIdx.z;
   const int32_t ts = seq_start(g, s), te = seq_end(g, s);
@@ -48,6 +52,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geom g, const int3
     for (int b = threadIdx.x; b < i; b += kRouteThreads)
       if (hist[b]) atomicAdd(counts + bucket_of(g, gk, s, b), hist[b]);
   } else {
+  {
+    const int64_t bk = bucket_of(g, gk, s, i - 1);
+    const int32_t t1 = __ldg(tile_off + bk + 1);
+    for (int32_t tt = __ldg(tile_off + bk) + threadIdx.x; tt < t1; tt += kRouteThreads) tile_bucket[tt] = (int32_t)bk;
+  }
   for (int b = threadIdx.x; b < i; b += kRouteThreads) {
     const int c = hist[b];
     base[b] = c ? atomicAdd(cursors + bucket_of(g, gk, s, b), c) : 0;
@@ -118,13 +127,13 @@ cudaError_t launch_route_tiles(const Geom& g, const int32_t* sel, const Work& w,
   e = cudaFuncSetAttribute(route_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(g.MB, g.num_seqs, g.Hkv);
-  route_kernel<false><<<grid, kRouteThreads, smem, st>>>(g, sel, w.counts, w.cursors, w.rows);
+  route_kernel<false><<<grid, kRouteThreads, smem, st>>>(g, sel, w.counts, w.cursors, w.rows, w.tile_off, w.tile_bucket);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   route_scan_kernel<<<1, kScanThreads, 0, st>>>(g.nbk, tile_m, w.counts, w.offsets, w.cursors, w.tile_off);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  route_kernel<true><<<grid, kRouteThreads, smem, st>>>(g, sel, w.counts, w.cursors, w.rows);
+  route_kernel<true><<<grid, kRouteThreads, smem, st>>>(g, sel, w.counts, w.cursors, w.rows, w.tile_off, w.tile_bucket);
   return cudaGetLastError();
 }
 
