@@ -51,6 +51,28 @@ constexpr uint32_t kColO = 256;    // O of tile t at kColO + 128 t
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when a row max grows by more than 2^8
 
+// 2^x for a pair on the FMA pipe, for a share of the exponentials that would otherwise all
+// queue on the MUFU unit: x = j + f with j = rint(x) (the 1.5 * 2^23 rounding trick) and
+// f in [-0.5, 0.5]; 2^f from a degree-3 polynomial (relative error 7.5e-5; coefficients from
+// our own iteratively reweighted least-squares fit of 2^f on that interval), 2^j added into
+// the exponent field.  x is clamped to >= -126 so the exponent never wraps; below 2^-24 the
+// result only has to be negligible next to the row sum, as it is.
+constexpr int kPolyNum = 1, kPolyDen = 4;  // pairs (pair index mod kPolyDen) < kPolyNum use it
+__device__ __forceinline__ void exp2_poly2(float& p0, float& p1, float x0, float x1) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, r0, r1, f0, f1, q0, q1;
+  add2(t0, t1, x0, x1, kRound, kRound);
+  add2(r0, r1, t0, t1, -kRound, -kRound);
+  fma2(f0, f1, r0, r1, -1.f, -1.f, x0, x1);
+  fma2(q0, q1, f0, f1, 0.05517132207751274f, 0.05517132207751274f, 0.24261054396629333f, 0.24261054396629333f);
+  fma2(q0, q1, q0, q1, f0, f1, 0.6932609677314758f, 0.6932609677314758f);
+  fma2(q0, q1, q0, q1, f0, f1, 0.9999281167984009f, 0.9999281167984009f);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 struct AttnArgs {
   Geom g;
   const __nv_bfloat16* Q;
@@ -244,7 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int x = 0; x < 32; ++x) mv[x & 7] = fmaxf(mv[x & 7], __uint_as_float(sr[c][x]));
+          for (int x = 0; x < 32; x += 2)
+            mv[(x >> 1) & 7] = max3(mv[(x >> 1) & 7], __uint_as_float(sr[c][x]), __uint_as_float(sr[c][x + 1]));
       } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -274,27 +297,49 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(tO + c * 32, o);
         }
       }
-      // p = 2^(s*c2 - m); P (bf16 pairs) overwrites the first 64 S columns (S is in registers)
+      // p = 2^(s*c2 - m); P (bf16 pairs) overwrites the first 64 S columns (S is in registers).
+      // Unmasked chunks work on pairs with f32x2 arithmetic and send a share of the
+      // exponentials to the FMA pipe; the diagonal chunk keeps the plain scalar form.
       float rv[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) rv[q] = 0.f;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t pk[32];
+        if (!masked) {
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int c = 2 * cc + h2;
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int c = 2 * cc + h2;
 #pragma unroll
-          for (int x = 0; x < 32; x += 2) {
-            float p0 = ex2(fmaf(__uint_as_float(sr[c][x]), c2, -m));
-            float p1 = ex2(fmaf(__uint_as_float(sr[c][x + 1]), c2, -m));
-            if (masked) {
+            for (int x = 0; x < 32; x += 2) {
+              const int pi = x >> 1;
+              float u0, u1, p0, p1;
+              fma2(u0, u1, __uint_as_float(sr[c][x]), __uint_as_float(sr[c][x + 1]), c2, c2, -m, -m);
+              if (pi % kPolyDen < kPolyNum) {
+                exp2_poly2(p0, p1, u0, u1);
+              } else {
+                p0 = ex2(u0);
+                p1 = ex2(u1);
+              }
+              const int q = 2 * (pi & 3);
+              add2(rv[q], rv[q + 1], rv[q], rv[q + 1], p0, p1);
+              pk[16 * h2 + pi] = pack_bf16x2(p0, p1);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int c = 2 * cc + h2;
+#pragma unroll
+            for (int x = 0; x < 32; x += 2) {
+              float p0 = ex2(fmaf(__uint_as_float(sr[c][x]), c2, -m));
+              float p1 = ex2(fmaf(__uint_as_float(sr[c][x + 1]), c2, -m));
               if (c * 32 + x >= lim) p0 = 0.f;
               if (c * 32 + x + 1 >= lim) p1 = 0.f;
+              rv[x & 7] += p0;
+              rv[(x & 7) + 1] += p1;
+              pk[16 * h2 + (x >> 1)] = pack_bf16x2(p0, p1);
             }
-            rv[x & 7] += p0;
-            rv[(x & 7) + 1] += p1;
-            pk[16 * h2 + (x >> 1)] = pack_bf16x2(p0, p1);
           }
         }
         tmem_st32(tP + cc * 32, pk);
