@@ -81,7 +81,7 @@ struct AttnArgs {
   const int32_t* tile_off;
   const int32_t* tile_bucket;
   const int32_t* rows;
-  float* part_o;
+  __half* part_o;
   float* part_lse;
   __nv_bfloat16* O;
   float* LSE;
@@ -401,29 +401,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (r < T_.nrows) a.part_lse[e] = lse_row;
       }
       if constexpr (!kOwn) {
-        // Each thread stages its own row (fp32; rows padded by 16 bytes so the row-per-thread
-        // 16-byte writes spread over the banks) and hands it to the TMA engine as one bulk
-        // copy to the row's partial slot.  The copies drain to memory on their own; the thread
-        // only waits until the engine has read the staged row.  Tile 0's warps stage in the Q
-        // and K buffers (free: the O barrier implies every QK^T MMA completed); tile 1's
-        // warps, whose O barrier follows the last MMA of the CTA, continue into the V buffers.
-        constexpr int kStgRow = D + 4;
-        static_assert(8 * 32 * kStgRow * 4 <= L::kBar && 4 * 32 * kStgRow * 4 <= L::kV0, "staging rows");
-        float* srow = reinterpret_cast<float*>(smem + L::kQ) + (warp * 32 + lane) * kStgRow;
+        // The normalised partial row goes out in fp16 (its rounding, at most 2^-11 of |O| per
+        // element, is far below the bf16 rounding of the final output).  Each thread stages its
+        // own row (rows padded by 16 bytes so the row-per-thread 16-byte writes spread over the
+        // banks) and hands it to the TMA engine as one bulk copy to the row's partial slot.
+        // The copies drain to memory on their own; the thread only waits until the engine has
+        // read the staged row.  Tile 0's warps stage in the Q and K buffers (free: the O
+        // barrier implies every QK^T MMA completed); tile 1's warps, whose O barrier follows
+        // the last MMA of the CTA, continue into the V buffers.
+        constexpr int kStgBytes = D * 2 + 16;
+        static_assert(8 * 32 * kStgBytes <= L::kBar && 4 * 32 * kStgBytes <= L::kV0, "staging rows");
+        uint8_t* srow = smem + L::kQ + (warp * 32 + lane) * kStgBytes;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
+          uint32_t hv[16];
 #pragma unroll
-          for (int x = 0; x < 32; x += 4)
-            *reinterpret_cast<float4*>(srow + c * 32 + x) =
-                make_float4(__uint_as_float(o[x]) * scale_row, __uint_as_float(o[x + 1]) * scale_row,
-                            __uint_as_float(o[x + 2]) * scale_row, __uint_as_float(o[x + 3]) * scale_row);
+          for (int x = 0; x < 32; x += 2) {
+            const __half2 h2v = __floats2half2_rn(__uint_as_float(o[x]) * scale_row, __uint_as_float(o[x + 1]) * scale_row);
+            hv[x >> 1] = *reinterpret_cast<const uint32_t*>(&h2v);
+          }
+#pragma unroll
+          for (int x = 0; x < 16; x += 4)
+            *reinterpret_cast<uint4*>(srow + c * 64 + x * 4) = make_uint4(hv[x], hv[x + 1], hv[x + 2], hv[x + 3]);
         }
         if (e >= 0) {
           fence_proxy_async_smem();
-          bulk_store_s2g(a.part_o + (int64_t)e * D, smem_u32(srow), D * 4);
+          bulk_store_s2g(a.part_o + (int64_t)e * D, smem_u32(srow), D * 2);
           bulk_commit();
           bulk_wait_read_all();
         }
@@ -440,12 +446,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             __uint_as_float(o[x + 2]) * scale_row, __uint_as_float(o[x + 3]) * scale_row);
         }
         __syncwarp();
-        // eight rows at a time, so their partial rows are all in flight together
-        constexpr int kU = 8;
+        // Eight rows at a time, so their partial rows are all in flight together.  Lane l
+        // covers the column pairs (64 p + 2 l, 64 p + 2 l + 1): fp16 partial pairs and bf16
+        // output pairs move in 128-byte warp-wide accesses.
+        constexpr int kU = 8, kPP = D / 64;
         for (int rr0 = 0; rr0 < 32; rr0 += kU) {
           int64_t qr[kU];
           int npr[kU];
-          float acc[kU][D / 32];
+          float acc[kU][kPP][2];
           int npmax = 0;
 #pragma unroll
           for (int u = 0; u < kU; ++u) {
@@ -453,11 +461,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             npr[u] = __shfl_sync(0xffffffffu, np, rr0 + u);
             npmax = max(npmax, npr[u]);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) acc[u][c] = *stg_at(rr0 + u, c * 32 + lane);
+            for (int pp = 0; pp < kPP; ++pp) {
+              const float2 v = *reinterpret_cast<const float2*>(stg_at(rr0 + u, pp * 64 + 2 * lane));
+              acc[u][pp][0] = v.x;
+              acc[u][pp][1] = v.y;
+            }
           }
           // partials two at a time: the loads of both are in flight together
           for (int q = 0; q < npmax; q += 2) {
-            float tmp[2][kU][D / 32];
+            __half2 tmp[2][kU][kPP];
             float wv[2];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
@@ -467,9 +479,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int u = 0; u < kU; ++u) {
                 const int32_t pq = __shfl_sync(0xffffffffu, pv, rr0 + u);
-                const float* src = a.part_o + (int64_t)pq * D + lane;
+                const __half2* src = reinterpret_cast<const __half2*>(a.part_o + (int64_t)pq * D) + lane;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) tmp[h2][u][c] = qq < npr[u] ? __ldg(src + c * 32) : 0.f;
+                for (int pp = 0; pp < kPP; ++pp)
+                  tmp[h2][u][pp] = qq < npr[u] ? __ldg(src + pp * 32) : __half2{};
               }
             }
 #pragma unroll
@@ -479,15 +492,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float wgt = __shfl_sync(0xffffffffu, wv[h2], rr0 + u);
                 if (q + h2 < npr[u])
 #pragma unroll
-                  for (int c = 0; c < D / 32; ++c) acc[u][c] = fmaf(wgt, tmp[h2][u][c], acc[u][c]);
+                  for (int pp = 0; pp < kPP; ++pp) {
+                    const float2 f = __half22float2(tmp[h2][u][pp]);
+                    acc[u][pp][0] = fmaf(wgt, f.x, acc[u][pp][0]);
+                    acc[u][pp][1] = fmaf(wgt, f.y, acc[u][pp][1]);
+                  }
               }
           }
 #pragma unroll
           for (int u = 0; u < kU; ++u) {
             if (qr[u] < 0) continue;
-            __nv_bfloat16* dst = a.O + qr[u] * D + lane;
+            __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.O + qr[u] * D) + lane;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) dst[c * 32] = __float2bfloat16_rn(acc[u][c]);
+            for (int pp = 0; pp < kPP; ++pp) dst[pp * 32] = __floats2bfloat162_rn(acc[u][pp][0], acc[u][pp][1]);
           }
         }
       }
@@ -512,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int64_t pq = qrow * (g.k - 1) + q;
             prefetch_l2(a.part_lse + pq);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) prefetch_l2(a.part_o + pq * D + c * 32);
+            for (int c = 0; c < D / 64; ++c) prefetch_l2(a.part_o + pq * D + c * 64);
           }
       }
     }

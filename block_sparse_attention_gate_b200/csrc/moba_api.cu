@@ -123,7 +123,7 @@ size_t carve(const moba::Geom& g, char* base, moba::Work* w) {
   x.tile_off = (int32_t*)take(sizeof(int32_t) * (size_t)(g.nbk + 1));
   x.tile_bucket = (int32_t*)take(sizeof(int32_t) * (size_t)moba::past_tiles(g));
   x.rows = (int32_t*)take(sizeof(int32_t) * (size_t)g.R);
-  x.part_o = (float*)take(sizeof(float) * (size_t)g.R * g.D);
+  x.part_o = (__half*)take(sizeof(__half) * (size_t)g.R * g.D);
   x.part_lse = (float*)take(sizeof(float) * (size_t)g.R);
   x.kbar = (float*)take(sizeof(float) * (size_t)g.num_seqs * g.MB * g.Hkv * g.D);
   x.sel = (int32_t*)take(sizeof(int32_t) * (size_t)g.T * g.Hq * g.k);

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace moba {
@@ -60,7 +61,7 @@ struct Work {
   int32_t* tile_off;  // [nbk + 1] exclusive scan of per-bucket tile counts
   int32_t* tile_bucket;  // [past_tiles(g)] bucket of each past-attention tile
   int32_t* rows;      // [R] routed partial ids, grouped by bucket
-  float* part_o;      // [R, D] normalised partial outputs
+  __half* part_o;     // [R, D] normalised partial outputs (fp16)
   float* part_lse;    // [R] partial log-sum-exp
   float* kbar;        // [num_seqs, MB, Hkv, D] (used by moba_fwd when the caller passes none)
   __nv_bfloat16* kbar_hi;  // [num_seqs, MB, Hkv, D] bf16 rn(Kbar) for the tensor-core gate
