@@ -77,7 +77,6 @@ struct AttnArgs {
   Geom g;
   const __nv_bfloat16* Q;
   const int32_t* sel;
-  const int32_t* offsets;
   const int32_t* tile_off;
   const int32_t* tile_bucket;
   const int32_t* rows;
@@ -131,19 +130,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t key0;
   TileInfo ti[2];
   if constexpr (!kOwn) {
-    const int32_t total = __ldg(a.tile_off + g.nbk);
+    // The routed rows are laid out tile by tile (kPastTileRows slots per tile, -1 in the
+    // slots past a bucket's last row), so a tile needs only its bucket and its own slots.
     const int32_t tile = (int32_t)blockIdx.x;
+    const int32_t total = __ldg(a.tile_off + g.nbk);
+    const int64_t lo = __ldg(a.tile_bucket + tile);  // in bounds for every launched tile
     if (tile >= total) return;
-    const int64_t lo = __ldg(a.tile_bucket + tile);  // this tile's bucket
     const int32_t b = (int32_t)(lo % g.MB);
     s = (int)((lo / g.MB) % g.num_seqs);
     gk = (int)(lo / ((int64_t)g.MB * g.num_seqs));
-    const int32_t rs = __ldg(a.offsets + lo) + (tile - __ldg(a.tile_off + lo)) * (2 * kRows);
-    const int32_t re = __ldg(a.offsets + lo + 1);
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      ti[t].row_start = rs + t * kRows;
-      ti[t].nrows = max(0, min(kRows, re - ti[t].row_start));
+      ti[t].row_start = tile * kPastTileRows + t * kRows;
+      ti[t].nrows = kRows;  // empty slots hold -1
       ti[t].diag = 1 << 30;
       ti[t].qrow_base = 0; ti[t].q0 = 0; ti[t].h = 0;
     }
@@ -189,6 +188,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     key0 = ts + i_blk * g.bs;
   }
 
+  // ------------------------------------------------------------- early loads
+  // Past mode: the softmax threads look up their routed rows and start the Q gather before
+  // the setup below.
+  int32_t e = -1;  // past mode: this thread's partial id (-1: empty slot)
+  if (!kOwn && warp < 8) {
+    const int t = warp >> 2, r = tid & (kRows - 1);
+    {
+      e = __ldg(a.rows + ti[t].row_start + r);
+      const int64_t qrow = e >= 0 ? e / (g.k - 1) : -1;
+      const __nv_bfloat16* src = qrow >= 0 ? a.Q + qrow * D : a.Q;
+      const uint32_t nb = qrow >= 0 ? 16u : 0u;  // zeros for empty slots
+      const uint32_t sQ = smem_u32(smem + L::kQ + t * L::kTile);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) cp_async_16(sQ + sw128_offset(r, c, kRows), src + c * 8, nb);
+    }
+  }
+  auto load_k = [&](int j) {  // K of chunk j into stage j & 1 (TMA producer)
+    const int st = j & 1;
+    const int tok = key0 + j * kBN;
+    mbar_expect_tx(&bars[kKFull0 + st], L::kTile);
+#pragma unroll
+    for (int hh = 0; hh < D / 64; ++hh)
+      tma_load_3d(smem + L::kK0 + st * L::kTile + hh * kRows * 128, &tmK, &bars[kKFull0 + st], hh * 64, gk, tok);
+  };
+  auto load_v = [&](int j) {
+    const int st = j & 1;
+    const int tok = key0 + j * kBN;
+    mbar_expect_tx(&bars[kVFull0 + st], L::kTile);
+#pragma unroll
+    for (int hh = 0; hh < D / 64; ++hh)
+      tma_load_3d(smem + L::kV0 + st * L::kTile + hh * kRows * 128, &tmV, &bars[kVFull0 + st], hh * 64, gk, tok);
+  };
+
   // ------------------------------------------------------------- setup
   if (warp == 9) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -220,22 +252,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = warp >> 2;           // tile
     const int r = tid & (kRows - 1);   // row = TMEM lane
     const TileInfo& T_ = ti[t];
-    int64_t qrow = -1;
-    int32_t e = -1;
-    if (r < T_.nrows) {
-      if constexpr (!kOwn) {
-        e = __ldg(a.rows + T_.row_start + r);
-        qrow = e / (g.k - 1);
-      } else {
-        qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
-      }
-    }
-    if constexpr (!kOwn) {  // gather this row of Q into tile t (zeros for padding rows)
-      const __nv_bfloat16* src = qrow >= 0 ? a.Q + qrow * D : a.Q;
-      const uint32_t nb = qrow >= 0 ? 16u : 0u;
-      const uint32_t sQ = smem_u32(smem + L::kQ + t * L::kTile);
-#pragma unroll
-      for (int c = 0; c < D / 8; ++c) cp_async_16(sQ + sw128_offset(r, c, kRows), src + c * 8, nb);
+    int64_t qrow = -1;  // own mode: this row's (token, head) row of Q, O and LSE
+    if (kOwn && r < T_.nrows) qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
+    if constexpr (!kOwn) {  // this row's Q gather (issued before the setup) has landed
       cp_async_wait_all();
       fence_proxy_async_smem();
       mbar_arrive(&bars[kQFull]);
@@ -398,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         scale_row = w_self * inv_l * inv_w;
         if (r < T_.nrows) a.LSE[qrow] = M + __logf(sumw);
       } else {
-        if (r < T_.nrows) a.part_lse[e] = lse_row;
+        if (e >= 0) a.part_lse[e] = lse_row;
       }
       if constexpr (!kOwn) {
         // The normalised partial row goes out in fp16 (its rounding, at most 2^-11 of |O| per
@@ -550,19 +569,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int j = 0; j < nchunks && ok; ++j) {
         const int st = j & 1, u = j >> 1;
-        const int tok = key0 + j * kBN;
         if (u > 0) ok = mbar_wait(&bars[kKEmpty0 + st], (u - 1) & 1, g.err);
         if (!ok) break;
-        mbar_expect_tx(&bars[kKFull0 + st], L::kTile);
-#pragma unroll
-        for (int hh = 0; hh < D / 64; ++hh)
-          tma_load_3d(smem + L::kK0 + st * L::kTile + hh * kRows * 128, &tmK, &bars[kKFull0 + st], hh * 64, gk, tok);
+        load_k(j);
         if (u > 0) ok = mbar_wait(&bars[kVEmpty0 + st], (u - 1) & 1, g.err);
         if (!ok) break;
-        mbar_expect_tx(&bars[kVFull0 + st], L::kTile);
-#pragma unroll
-        for (int hh = 0; hh < D / 64; ++hh)
-          tma_load_3d(smem + L::kV0 + st * L::kTile + hh * kRows * 128, &tmV, &bars[kVFull0 + st], hh * 64, gk, tok);
+        load_v(j);
       }
     }
   } else if (warp == 9) {
@@ -648,7 +660,7 @@ cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16
   }
   e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
-  AttnArgs a{g, Q, sel, w.offsets, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, O, LSE, head_pairs};
+  AttnArgs a{g, Q, sel, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, O, LSE, head_pairs};
   const int smem = Layout<D>::kAlloc;
   e = cudaFuncSetAttribute(attn_tc_kernel<D, kOwn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

@@ -118,11 +118,10 @@ size_t carve(const moba::Geom& g, char* base, moba::Work* w) {
   };
   moba::Work x;
   x.counts = (int32_t*)take(sizeof(int32_t) * (size_t)g.nbk);
-  x.offsets = (int32_t*)take(sizeof(int32_t) * (size_t)(g.nbk + 1));
   x.cursors = (int32_t*)take(sizeof(int32_t) * (size_t)g.nbk);
   x.tile_off = (int32_t*)take(sizeof(int32_t) * (size_t)(g.nbk + 1));
   x.tile_bucket = (int32_t*)take(sizeof(int32_t) * (size_t)moba::past_tiles(g));
-  x.rows = (int32_t*)take(sizeof(int32_t) * (size_t)g.R);
+  x.rows = (int32_t*)take(sizeof(int32_t) * (size_t)moba::past_tiles(g) * moba::kPastTileRows);
   x.part_o = (__half*)take(sizeof(__half) * (size_t)g.R * g.D);
   x.part_lse = (float*)take(sizeof(float) * (size_t)g.R);
   x.kbar = (float*)take(sizeof(float) * (size_t)g.num_seqs * g.MB * g.Hkv * g.D);

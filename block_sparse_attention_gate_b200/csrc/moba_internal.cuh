@@ -56,11 +56,10 @@ __device__ __forceinline__ int find_seq(const Geom& g, int32_t t) {
 // Workspace carve-up (device pointers; every region 256-byte aligned).
 struct Work {
   int32_t* counts;    // [nbk] rows routed to each (kv head, sequence, block) bucket
-  int32_t* offsets;   // [nbk + 1] exclusive scan of counts
   int32_t* cursors;   // [nbk] scatter cursors
   int32_t* tile_off;  // [nbk + 1] exclusive scan of per-bucket tile counts
   int32_t* tile_bucket;  // [past_tiles(g)] bucket of each past-attention tile
-  int32_t* rows;      // [R] routed partial ids, grouped by bucket
+  int32_t* rows;      // [past_tiles(g) * kPastTileRows] routed partial ids, tile by tile (-1: empty)
   __half* part_o;     // [R, D] normalised partial outputs (fp16)
   float* part_lse;    // [R] partial log-sum-exp
   float* kbar;        // [num_seqs, MB, Hkv, D] (used by moba_fwd when the caller passes none)

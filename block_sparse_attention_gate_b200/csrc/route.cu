@@ -1,8 +1,10 @@
 // Query-to-block routing (the "organise the data" step of the youleyou.com article,
 // section "PyTorch实现关键要点", done MoE-style): every (token, query head, slot >= 1)
 // whose selected past block is b joins bucket (kv head g, sequence s, block b).
-// Three passes: per-CTA shared-memory histograms flushed to global counts; one-CTA
-// exclusive scans (rows and attention tiles per bucket); scatter of partial ids.
+// Three passes: per-CTA shared-memory histograms flushed to global counts; a one-CTA
+// exclusive scan of the attention tiles per bucket; scatter of partial ids.  The routed
+// rows are laid out tile by tile: bucket b owns slots [tile_off[b], tile_off[b+1]) * tile_m,
+// its rows first and -1 in the rest, so an attention tile reads only its own slots.
 //
 // A partial id is e = (t * Hq + h) * (k - 1) + (slot - 1); it indexes the partial
 // output buffers directly, so the order inside a bucket does not affect any result.
@@ -18,8 +20,9 @@ __device__ __forceinline__ int64_t bucket_of(const Geom& g, int gk, int s, int32
 }
 
 // grid (MB, num_seqs, Hkv): CTA = query block i of sequence s, KV head g
-// The scatter pass also fills the tile -> bucket table: CTA (i, s, g) writes the tiles of
-// bucket (g, s, i - 1), so every bucket that can hold rows is covered exactly once.
+// The scatter pass also fills, for bucket (g, s, i - 1), the tile -> bucket table and the
+// empty slots of its last tile (CTA (i, s, g) exists for every bucket that can hold rows, so
+// each such bucket is covered exactly once).
 template <bool kScatter>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geom g, const int32_t* __restrict__ sel,
                                                             int32_t* __restrict__ counts,
@@ -54,8 +57,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geom g, const int3
   } else {
   {
     const int64_t bk = bucket_of(g, gk, s, i - 1);
-    const int32_t t1 = __ldg(tile_off + bk + 1);
-    for (int32_t tt = __ldg(tile_off + bk) + threadIdx.x; tt < t1; tt += kRouteThreads) tile_bucket[tt] = (int32_t)bk;
+    const int32_t t0 = __ldg(tile_off + bk), t1 = __ldg(tile_off + bk + 1);
+    for (int32_t tt = t0 + threadIdx.x; tt < t1; tt += kRouteThreads) tile_bucket[tt] = (int32_t)bk;
+    const int64_t slot_end = (int64_t)t1 * kPastTileRows;
+    for (int64_t sl = (int64_t)t0 * kPastTileRows + __ldg(counts + bk) + threadIdx.x; sl < slot_end; sl += kRouteThreads)
+      rows[sl] = -1;
   }
   for (int b = threadIdx.x; b < i; b += kRouteThreads) {
     const int c = hist[b];
@@ -78,43 +84,33 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geom g, const int3
   }
 }
 
-// Exclusive scans of the bucket row counts and of their tile counts (tile = tile_m rows).
+// Exclusive scan of the bucket tile counts (tile = tile_m rows); each bucket's scatter
+// cursor starts at its first slot.
 __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(int64_t nbk, int tile_m,
                                                                 const int32_t* __restrict__ counts,
-                                                                int32_t* __restrict__ offsets,
                                                                 int32_t* __restrict__ cursors,
                                                                 int32_t* __restrict__ tile_off) {
-  __shared__ int64_t sr[kScanThreads], st[kScanThreads];
+  __shared__ int64_t st[kScanThreads];
   const int tid = threadIdx.x;
   const int64_t per = (nbk + kScanThreads - 1) / kScanThreads;
   const int64_t lo = min(nbk, per * tid), hi = min(nbk, lo + per);
-  int64_t r = 0, tl = 0;
-  for (int64_t j = lo; j < hi; ++j) {
-    r += counts[j];
-    tl += (counts[j] + tile_m - 1) / tile_m;
-  }
-  sr[tid] = r;
+  int64_t tl = 0;
+  for (int64_t j = lo; j < hi; ++j) tl += (counts[j] + tile_m - 1) / tile_m;
   st[tid] = tl;
   __syncthreads();
   for (int off = 1; off < kScanThreads; off <<= 1) {
-    int64_t a = tid >= off ? sr[tid - off] : 0, b = tid >= off ? st[tid - off] : 0;
+    const int64_t b = tid >= off ? st[tid - off] : 0;
     __syncthreads();
-    sr[tid] += a;
     st[tid] += b;
     __syncthreads();
   }
-  int64_t rr = sr[tid] - r, tt = st[tid] - tl;
+  int64_t tt = st[tid] - tl;
   for (int64_t j = lo; j < hi; ++j) {
-    offsets[j] = (int32_t)rr;
-    cursors[j] = (int32_t)rr;
+    cursors[j] = (int32_t)(tt * tile_m);
     tile_off[j] = (int32_t)tt;
-    rr += counts[j];
     tt += (counts[j] + tile_m - 1) / tile_m;
   }
-  if (tid == kScanThreads - 1) {
-    offsets[nbk] = (int32_t)sr[tid];
-    tile_off[nbk] = (int32_t)st[tid];
-  }
+  if (tid == kScanThreads - 1) tile_off[nbk] = (int32_t)st[tid];
 }
 
 cudaError_t launch_route_tiles(const Geom& g, const int32_t* sel, const Work& w, int tile_m,
@@ -130,7 +126,7 @@ cudaError_t launch_route_tiles(const Geom& g, const int32_t* sel, const Work& w,
   route_kernel<false><<<grid, kRouteThreads, smem, st>>>(g, sel, w.counts, w.cursors, w.rows, w.tile_off, w.tile_bucket);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  route_scan_kernel<<<1, kScanThreads, 0, st>>>(g.nbk, tile_m, w.counts, w.offsets, w.cursors, w.tile_off);
+  route_scan_kernel<<<1, kScanThreads, 0, st>>>(g.nbk, tile_m, w.counts, w.cursors, w.tile_off);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   route_kernel<true><<<grid, kRouteThreads, smem, st>>>(g, sel, w.counts, w.cursors, w.rows, w.tile_off, w.tile_bucket);

@@ -35,7 +35,7 @@ def test_sizes_are_host_computations():
     assert p.kbar_elems == 512 * 8 * 128
     ws = p.workspace_bytes
     R = (1 << 20) * 32 * 2
-    assert ws >= R * 128 * 4 + R * 8 + (1 << 20) * 32 * 3 * 4
+    assert ws >= R * 128 * 2 + R * 8 + (1 << 20) * 32 * 3 * 4  # fp16 partial rows, LSE, row ids, sel
     # varlen: MB follows the longest sequence
     q = mb.MobaParams.__new__(mb.MobaParams)
     cu = np.array([0, 131072, 196608, 229376, 245760], dtype=np.int32)
