@@ -1,13 +1,14 @@
 // MoBA block attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
 //
 // Two modes share one kernel body:
-//   past : a CTA takes a tile of up to 128 routed query rows of one bucket (KV head g,
+//   past : a CTA takes two tiles of 128 routed query rows of one bucket (KV head g,
 //          sequence s, past block b), attends the whole block (bs keys; a past block is
-//          complete and fully visible) and writes normalised fp32 partials + LSE.
-//   own  : a CTA takes 128 consecutive tokens of one query head inside one block, attends
-//          the block's keys up to the diagonal (causal mask on the diagonal chunk), then
-//          merges the past partials of every row by online softmax and writes O (bf16) and
-//          LSE.
+//          complete and fully visible) and writes normalised partials (fp16) + LSE (fp32).
+//   own  : a CTA takes two tiles of 128 tokens (two heads, or two consecutive tiles of one
+//          head) inside one block.  Each row's past partials are merged FIRST: they become
+//          the starting state (m, l, O) of the online softmax, which then runs over the
+//          block's keys up to the diagonal (causal mask on the diagonal chunk) and ends with
+//          the final O (bf16) and LSE.
 // (youleyou.com, "Kimi发布MoBA突破性实现无限上下文", section "PyTorch实现关键要点": attention
 // runs on the own block and on the selected blocks separately and the results are merged by
 // online softmax; zhuoshang.net, "MoBA是什么？…", section "MoBA的技术原理": causal mask inside
@@ -21,8 +22,7 @@
 // The tensor core works on one tile while the other tile's softmax runs.
 // Warp roles: warps 0-3 softmax + epilogue of tile 0, warps 4-7 of tile 1, warp 8 TMA
 // producer (K/V chunks, two stages), warp 9 TMEM owner + MMA issuer (the whole warp runs the
-// issue loop; one elected lane issues each tcgen05.mma), warps 10-11 register donors (in own
-// mode they also prefetch the merge inputs into L2).
+// issue loop; one elected lane issues each tcgen05.mma), warps 10-11 register donors.
 #include <cudaTypedefs.h>
 #include <float.h>
 
@@ -49,6 +49,7 @@ constexpr uint32_t kColS = 0;      // S of tile t at kColS + 128 t
 constexpr uint32_t kColP = 0;      // P of tile t (bf16 pairs) aliased at S + 0 .. S + 63
 constexpr uint32_t kColO = 256;    // O of tile t at kColO + 128 t
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when a row max grows by more than 2^8
 
 // 2^x for a pair on the FMA pipe, for a share of the exponentials that would otherwise all
@@ -265,6 +266,67 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_off + kColO + t * 128;
     const float c2 = g.scale_log2;
     float m = -INFINITY, l = 0.f;
+    if constexpr (kOwn) {
+      // Merge first: the row's past partials (normalised O_q and LSE_q, written by the
+      // past-block attention before this kernel runs) become the starting state of the
+      // online softmax, in its log2 units: m = max_q LSE_q log2(e), w_q = 2^(LSE_q log2(e) - m),
+      // l = sum_q w_q, O = sum_q w_q O_q (the past keys' share of sum_k 2^(s_k c2 - m) v_k).
+      // The own block's chunks then continue the same online softmax; the O accumulator is
+      // written here, before the first PV MMA (which accumulates onto it).
+      int np = 0;
+      int32_t pe[kMaxTopK - 1];
+      float pl[kMaxTopK - 1];
+      if (qrow >= 0) {
+        int32_t bsel[kMaxTopK - 1];
+#pragma unroll
+        for (int q = 0; q < kMaxTopK - 1; ++q) bsel[q] = q + 1 < g.k ? __ldg(a.sel + qrow * g.k + q + 1) : -1;
+#pragma unroll
+        for (int q = 0; q < kMaxTopK - 1; ++q)
+          if (bsel[q] >= 0 && bsel[q] < i_blk) pe[np++] = (int32_t)(qrow * (g.k - 1) + q);
+#pragma unroll
+        for (int q = 0; q < kMaxTopK - 1; ++q)
+          if (q < np) pl[q] = __ldg(a.part_lse + pe[q]) * kLog2e;
+      }
+      for (int q = 0; q < np; ++q) m = fmaxf(m, pl[q]);
+      const int npmax = __reduce_max_sync(0xffffffffu, np);
+      for (int q0 = 0; q0 < npmax || q0 == 0; q0 += 2) {  // warp-uniform: TMEM access is per warp
+        uint4 hv[2][D / 8];
+        float w[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int q = q0 + h2;
+          const bool have = q < np;
+          w[h2] = have ? ex2(pl[q] - m) : 0.f;
+          const uint4* src = reinterpret_cast<const uint4*>(a.part_o + (int64_t)(have ? pe[q] : 0) * D);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) hv[h2][c] = have ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+        }
+        l += w[0] + w[1];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          if (q0 > 0) {
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = 0u;
+          }
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const __half2* hp = reinterpret_cast<const __half2*>(&hv[h2][c * 4]);
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              const float2 f = __half22float2(hp[x]);
+              o[2 * x] = __float_as_uint(fmaf(w[h2], f.x, __uint_as_float(o[2 * x])));
+              o[2 * x + 1] = __float_as_uint(fmaf(w[h2], f.y, __uint_as_float(o[2 * x + 1])));
+            }
+          }
+          tmem_st32(tO + c * 32, o);
+        }
+        tmem_wait_st();
+      }
+    }
     for (int j = 0; j < nchunks && ok; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull0 + t], j & 1, g.err));
       if (!ok) break;
@@ -299,9 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // running max: rescale the TMEM accumulator only when it grows by more than 2^8
       // (p <= 256 otherwise, harmless in fp32 sums and bf16 P).  At this point the previous
       // PV of this tile has completed: the MMA that produced this S was issued after it.
-      if (j == 0) {
+      if (!kOwn && j == 0) {
         m = mx;
-      } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
+      } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {  // own mode: m may start at -inf
         const float m_new = fmaxf(m, mx);
         const float alpha = ex2(m - m_new);
         l *= alpha;
@@ -375,181 +437,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const float lse_row = (m + __log2f(l)) * kLn2;
-      // own mode: each warp stages its 32 rows (fp32, D columns) in shared memory that no MMA
-      // reads any more (this tile's Q buffer and one K stage: every QK^T MMA completed before
-      // the O barrier fired), then merges and writes whole rows cooperatively.  16-byte chunks
-      // of a staged row are XOR-swizzled by (row mod 8) to spread the row-per-thread writes
-      // over the banks.
-      const int wq = warp & 3;
-      float* stg = reinterpret_cast<float*>(smem + (wq < 2 ? L::kQ : L::kK0) + t * L::kTile + (wq & 1) * (L::kTile / 2));
-      auto stg_at = [&](int row, int col) -> float* {
-        return stg + row * D + ((((col >> 2) ^ (row & 7)) << 2) | (col & 3));
-      };
-      float scale_row = inv_l;
-      // own mode: merge weights of this row (own block and its past partials).  The loads
-      // are independent of one another (all slots, then all LSEs) and hit L2: warps 10-11
-      // pulled these lines in while the block attention ran.
-      float M = lse_row, inv_w = 1.f;
-      int32_t pe[kMaxTopK];
-      float pw[kMaxTopK];
-      int np = 0;
-      if constexpr (kOwn) {
-        if (r < T_.nrows) {
-          int32_t bsel[kMaxTopK - 1];
+      // Past mode: the normalised partial row (fp16: its rounding, at most 2^-11 of |O| per
+      // element, is far below the bf16 rounding of the final output) and its LSE, at the
+      // row's partial id.  Own mode: the final O row (bf16) and LSE: the past partials were
+      // merged in at the start.
+      // Each thread stages its own row (rows padded by 16 bytes so the row-per-thread 16-byte
+      // writes spread over the banks) and hands it to the TMA engine as one bulk copy.  The
+      // copies drain to memory on their own; the thread only waits until the engine has read
+      // the staged row.  Tile 0's warps stage in the Q and K buffers (free: the O barrier
+      // implies every QK^T MMA completed); tile 1's warps, whose O barrier follows the last
+      // MMA of the CTA, continue into the V buffers.
+      constexpr int kStgBytes = D * 2 + 16;
+      static_assert(8 * 32 * kStgBytes <= L::kBar && 4 * 32 * kStgBytes <= L::kV0, "staging rows");
+      uint8_t* srow = smem + L::kQ + (warp * 32 + lane) * kStgBytes;
 #pragma unroll
-          for (int q = 0; q < kMaxTopK - 1; ++q) bsel[q] = q + 1 < g.k ? __ldg(a.sel + qrow * g.k + q + 1) : -1;
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_wait_ld();
+        uint32_t hv[16];
 #pragma unroll
-          for (int q = 0; q < kMaxTopK - 1; ++q)
-            if (bsel[q] >= 0 && bsel[q] < i_blk) pe[np++] = (int32_t)(qrow * (g.k - 1) + q);
-#pragma unroll
-          for (int q = 0; q < kMaxTopK - 1; ++q)
-            if (q < np) pw[q] = __ldg(a.part_lse + pe[q]);
-        }
-        for (int q = 0; q < np; ++q) M = fmaxf(M, pw[q]);
-        const float w_self = __expf(lse_row - M);
-        float sumw = w_self;
-        for (int q = 0; q < np; ++q) {
-          pw[q] = __expf(pw[q] - M);
-          sumw += pw[q];
-        }
-        inv_w = 1.f / sumw;
-        for (int q = 0; q < np; ++q) pw[q] *= inv_w;
-        scale_row = w_self * inv_l * inv_w;
-        if (r < T_.nrows) a.LSE[qrow] = M + __logf(sumw);
-      } else {
-        if (e >= 0) a.part_lse[e] = lse_row;
-      }
-      if constexpr (!kOwn) {
-        // The normalised partial row goes out in fp16 (its rounding, at most 2^-11 of |O| per
-        // element, is far below the bf16 rounding of the final output).  Each thread stages its
-        // own row (rows padded by 16 bytes so the row-per-thread 16-byte writes spread over the
-        // banks) and hands it to the TMA engine as one bulk copy to the row's partial slot.
-        // The copies drain to memory on their own; the thread only waits until the engine has
-        // read the staged row.  Tile 0's warps stage in the Q and K buffers (free: the O
-        // barrier implies every QK^T MMA completed); tile 1's warps, whose O barrier follows
-        // the last MMA of the CTA, continue into the V buffers.
-        constexpr int kStgBytes = D * 2 + 16;
-        static_assert(8 * 32 * kStgBytes <= L::kBar && 4 * 32 * kStgBytes <= L::kV0, "staging rows");
-        uint8_t* srow = smem + L::kQ + (warp * 32 + lane) * kStgBytes;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-          uint32_t hv[16];
-#pragma unroll
-          for (int x = 0; x < 32; x += 2) {
-            const __half2 h2v = __floats2half2_rn(__uint_as_float(o[x]) * scale_row, __uint_as_float(o[x + 1]) * scale_row);
+        for (int x = 0; x < 32; x += 2) {
+          const float v0 = __uint_as_float(o[x]) * inv_l, v1 = __uint_as_float(o[x + 1]) * inv_l;
+          if constexpr (kOwn) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
+            hv[x >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
+          } else {
+            const __half2 h2v = __floats2half2_rn(v0, v1);
             hv[x >> 1] = *reinterpret_cast<const uint32_t*>(&h2v);
           }
-#pragma unroll
-          for (int x = 0; x < 16; x += 4)
-            *reinterpret_cast<uint4*>(srow + c * 64 + x * 4) = make_uint4(hv[x], hv[x + 1], hv[x + 2], hv[x + 3]);
         }
-        if (e >= 0) {
-          fence_proxy_async_smem();
-          bulk_store_s2g(a.part_o + (int64_t)e * D, smem_u32(srow), D * 2);
-          bulk_commit();
-          bulk_wait_read_all();
+#pragma unroll
+        for (int x = 0; x < 16; x += 4)
+          *reinterpret_cast<uint4*>(srow + c * 64 + x * 4) = make_uint4(hv[x], hv[x + 1], hv[x + 2], hv[x + 3]);
+      }
+      void* dst = nullptr;
+      if constexpr (kOwn) {
+        if (qrow >= 0) {
+          a.LSE[qrow] = lse_row;
+          dst = a.O + qrow * D;
         }
       } else {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int x = 0; x < 32; x += 4)
-            *reinterpret_cast<float4*>(stg_at(lane, c * 32 + x)) =
-                make_float4(__uint_as_float(o[x]) * scale_row, __uint_as_float(o[x + 1]) * scale_row,
-                            __uint_as_float(o[x + 2]) * scale_row, __uint_as_float(o[x + 3]) * scale_row);
-        }
-        __syncwarp();
-        // Eight rows at a time, so their partial rows are all in flight together.  Lane l
-        // covers the column pairs (64 p + 2 l, 64 p + 2 l + 1): fp16 partial pairs and bf16
-        // output pairs move in 128-byte warp-wide accesses.
-        constexpr int kU = 8, kPP = D / 64;
-        for (int rr0 = 0; rr0 < 32; rr0 += kU) {
-          int64_t qr[kU];
-          int npr[kU];
-          float acc[kU][kPP][2];
-          int npmax = 0;
-#pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            qr[u] = __shfl_sync(0xffffffffu, qrow, rr0 + u);
-            npr[u] = __shfl_sync(0xffffffffu, np, rr0 + u);
-            npmax = max(npmax, npr[u]);
-#pragma unroll
-            for (int pp = 0; pp < kPP; ++pp) {
-              const float2 v = *reinterpret_cast<const float2*>(stg_at(rr0 + u, pp * 64 + 2 * lane));
-              acc[u][pp][0] = v.x;
-              acc[u][pp][1] = v.y;
-            }
-          }
-          // partials two at a time: the loads of both are in flight together
-          for (int q = 0; q < npmax; q += 2) {
-            __half2 tmp[2][kU][kPP];
-            float wv[2];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int qq = q + h2;
-              const int32_t pv = qq < np ? pe[qq] : 0;
-              wv[h2] = qq < np ? pw[qq] : 0.f;
-#pragma unroll
-              for (int u = 0; u < kU; ++u) {
-                const int32_t pq = __shfl_sync(0xffffffffu, pv, rr0 + u);
-                const __half2* src = reinterpret_cast<const __half2*>(a.part_o + (int64_t)pq * D) + lane;
-#pragma unroll
-                for (int pp = 0; pp < kPP; ++pp)
-                  tmp[h2][u][pp] = qq < npr[u] ? __ldg(src + pp * 32) : __half2{};
-              }
-            }
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-              for (int u = 0; u < kU; ++u) {
-                const float wgt = __shfl_sync(0xffffffffu, wv[h2], rr0 + u);
-                if (q + h2 < npr[u])
-#pragma unroll
-                  for (int pp = 0; pp < kPP; ++pp) {
-                    const float2 f = __half22float2(tmp[h2][u][pp]);
-                    acc[u][pp][0] = fmaf(wgt, f.x, acc[u][pp][0]);
-                    acc[u][pp][1] = fmaf(wgt, f.y, acc[u][pp][1]);
-                  }
-              }
-          }
-#pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            if (qr[u] < 0) continue;
-            __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.O + qr[u] * D) + lane;
-#pragma unroll
-            for (int pp = 0; pp < kPP; ++pp) dst[pp * 32] = __floats2bfloat162_rn(acc[u][pp][0], acc[u][pp][1]);
-          }
+        if (e >= 0) {
+          a.part_lse[e] = lse_row;
+          dst = a.part_o + (int64_t)e * D;
         }
       }
-    }
-  } else if (warp >= 10) {
-    // ========================================================= own mode: merge-input prefetch
-    // Warps 10-11 have no role in the attention itself.  In own mode they pull every row's
-    // merge inputs into L2 while the block attention runs (the past partials exist before
-    // this kernel starts): the chosen-block slots, then each past partial's LSE and O row.
-    if constexpr (kOwn) {
-      for (int rr = tid - 10 * 32; rr < 2 * kRows; rr += 64) {
-        const TileInfo& T_ = ti[rr / kRows];
-        const int r = rr % kRows;
-        if (r >= T_.nrows) continue;
-        const int64_t qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
-        int32_t bsel[kMaxTopK - 1];
-#pragma unroll
-        for (int q = 0; q < kMaxTopK - 1; ++q) bsel[q] = q + 1 < g.k ? __ldg(a.sel + qrow * g.k + q + 1) : -1;
-#pragma unroll
-        for (int q = 0; q < kMaxTopK - 1; ++q)
-          if (bsel[q] >= 0 && bsel[q] < i_blk) {
-            const int64_t pq = qrow * (g.k - 1) + q;
-            prefetch_l2(a.part_lse + pq);
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c) prefetch_l2(a.part_o + pq * D + c * 64);
-          }
+      if (dst) {
+        fence_proxy_async_smem();
+        bulk_store_s2g(dst, smem_u32(srow), D * 2);
+        bulk_commit();
+        bulk_wait_read_all();
       }
     }
   } else if (warp == 8) {
@@ -599,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk)
         mma_bf16_ts_warp(tmem + kColO + t * 128, tmem + kColS + t * kBN + kColP + kk * 8,
-                         sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
+                         sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), idO, (kOwn || j > 0 || kk > 0) ? 1u : 0u);
     };
     ok = mbar_wait_warp(&bars[kQFull], 0, g.err) && mbar_wait_warp(&bars[kKFull0], 0, g.err);
     if (ok) {
