@@ -7,7 +7,7 @@
 // query with the pooled keys, mask future blocks, top-k.)
 //
 // A CTA takes 128 consecutive tokens of one query head inside one query block i.  The
-// candidate blocks 0..i-1 are processed in chunks of up to 128: the chunk's pooled keys,
+// candidate blocks 0..i-1 are processed in chunks of up to 64: the chunk's pooled keys,
 // split into bf16 hi + lo parts (Kbar = hi + lo + O(2^-17 |Kbar|)), are staged by TMA and
 // S = Q hi^T + Q lo^T accumulates in fp32 TMEM (double-buffered).  Thread r reads row r
 // of S from TMEM and keeps a sorted running top-(k-1) list in registers.
@@ -24,15 +24,15 @@ namespace {
 
 constexpr int kThreads = 160;     // warps 0-3 epilogue, warp 4 TMA + MMA (whole warp)
 constexpr int kRows = 128;        // query rows per CTA
-constexpr int kCand = 128;        // candidate blocks per chunk
+constexpr int kCand = 64;         // candidate blocks per chunk (three CTAs per SM)
 constexpr int kBoxRows = 64;      // candidate rows per TMA box
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 128;
 
 template <int D>
 struct GLayout {
   static constexpr int kQ = 0;                       // [128 x D] bf16
-  static constexpr int kHi = kQ + kRows * D * 2;     // [128 x D] bf16
-  static constexpr int kLo = kHi + kCand * D * 2;    // [128 x D] bf16
+  static constexpr int kHi = kQ + kRows * D * 2;     // [kCand x D] bf16
+  static constexpr int kLo = kHi + kCand * D * 2;    // [kCand x D] bf16
   static constexpr int kBar = kLo + kCand * D * 2;
   static constexpr int kAlloc = kBar + 128 + 1024;
 };
@@ -46,7 +46,7 @@ __device__ __forceinline__ bool ranks_before(float sa, int32_t ba, float sb, int
 // kMaxM: compile-time capacity of the running top lists (>= top_k - 1), so the lists live
 // in registers; kLists of them take interleaved candidates to shorten the dependency chain.
 template <int D, int kMaxM, int kLists = (kMaxM <= 4 ? 4 : (kMaxM <= 8 ? 2 : 1))>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 3)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmHi,
                    const __grid_constant__ CUtensorMap tmLo, Geom g, int32_t* __restrict__ sel) {
   using L = GLayout<D>;
