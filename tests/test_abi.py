@@ -87,3 +87,15 @@ def test_empty_problem_is_a_no_op():
     p = mb.MobaParams(None, 2, 1, 64, 128, 3, num_seqs=1, max_seqlen=0)
     lib = mb.load()
     assert lib.moba_fwd(p.ref(), None, None, None, None, None, None, 0, None, None, None) == 0
+
+
+def test_host_staging_is_per_slot_group_sized():
+    # one slot holds one KV-head group's Q, K, V, O, LSE and that group's workspace
+    p = mb.MobaParams(None, 32, 8, 128, 2048, 3, num_seqs=1, max_seqlen=1 << 16)
+    one = mb.moba_host_staging_size(p, 1)
+    assert one > 0 and mb.moba_host_staging_size(p, 3) == 3 * one
+    T, G, D = 1 << 16, 4, 128
+    group_io = T * G * D * 2 * 2 + T * D * 2 * 2 + T * G * 4  # Q and O, K and V, LSE
+    g = mb.MobaParams(None, G, 1, D, 2048, 3, num_seqs=1, max_seqlen=T)
+    assert group_io + g.workspace_bytes <= one <= group_io + g.workspace_bytes + 8 * 256
+    assert mb.moba_host_staging_size(p, 0) == 0
