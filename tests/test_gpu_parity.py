@@ -37,6 +37,20 @@ SMALL = {
     "bs8192": synth.Workload("bs8192", [9000], 2, 1, 128, 8192, 2, seed=15, rope_theta=500000.0),
     # the largest top_k with more blocks than it
     "top16": synth.Workload("top16", [2560, 1100], 2, 2, 128, 128, 16, seed=16),
+    # top_k 6, 8 and 9 (at most 8 past blocks: the gate's two interleaved 8-slot lists), at
+    # head_dim 128 and 64
+    "k6_d128": synth.Workload("k6_d128", [2000, 1100], 4, 2, 128, 128, 6, seed=18,
+                              rope_theta=500000.0, plant=0.5),
+    "k8_d64": synth.Workload("k8_d64", [1700, 1300], 4, 1, 64, 128, 8, seed=19,
+                             rope_theta=10000.0),
+    "k9_d128": synth.Workload("k9_d128", [2300], 2, 2, 128, 128, 9, seed=20),
+    # more than 64 past blocks: the gate walks its candidates in several 64-block chunks
+    # through the double-buffered score accumulator (73 and 133 blocks)
+    "chunks_d128": synth.Workload("chunks_d128", [9300], 4, 2, 128, 128, 3, seed=23,
+                                  rope_theta=500000.0, plant=0.5),
+    "chunks_d64_k8": synth.Workload("chunks_d64_k8", [17000], 2, 1, 64, 128, 8, seed=24,
+                                    rope_theta=500000.0, plant=0.5),
+    "chunks_k16": synth.Workload("chunks_k16", [9000, 300], 2, 1, 128, 128, 16, seed=25),
     # many short sequences
     "many_seqs": synth.Workload("many_seqs", list(np.random.default_rng(17).integers(1, 300, 300)), 2, 1, 64,
                                 128, 3, seed=17),
