@@ -5,6 +5,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "moba.h"
 #include "moba_internal.cuh"
 #include "sm100.cuh"
@@ -134,7 +136,26 @@ size_t carve(const moba::Geom& g, char* base, moba::Work* w) {
 }
 
 constexpr int kMaxDevices = 64;
-int* g_err_ptr[kMaxDevices] = {};  // device address of g_moba_device_error, per device
+
+// Device address of a __device__ variable, looked up once per device (with that device
+// current) by the first caller; concurrent first callers on other host threads wait for it.
+// The host-side name of a __device__ variable is only a stand-in, never a device address.
+// The cached address belongs to the device's primary context: it is not valid after
+// cudaDeviceReset on that device.
+struct SymbolAddress {
+  std::once_flag once[kMaxDevices];
+  void* ptr[kMaxDevices] = {};
+  cudaError_t err[kMaxDevices] = {};
+};
+
+template <typename Sym>
+cudaError_t symbol_address(SymbolAddress& cache, int dev, const Sym& symbol, void** out) {
+  std::call_once(cache.once[dev], [&] { cache.err[dev] = cudaGetSymbolAddress(&cache.ptr[dev], symbol); });
+  *out = cache.ptr[dev];
+  return cache.err[dev];
+}
+
+SymbolAddress g_err_addr;  // g_moba_device_error
 
 // Checks that the current device is an sm_100 part and binds the device error word's
 // address (looked up once per device with that device current) into the geometry.
@@ -149,13 +170,10 @@ moba_status check_device(moba::Geom* g) {
   if (major != 10 || minor != 0)
     return fail(MOBA_ERR_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a", dev, major, minor);
   if (dev < 0 || dev >= kMaxDevices) return fail(MOBA_ERR_DEVICE, "device ordinal %d out of range", dev);
-  if (!g_err_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_moba_device_error);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
-    g_err_ptr[dev] = static_cast<int*>(p);
-  }
-  g->err = g_err_ptr[dev];
+  void* p = nullptr;
+  e = symbol_address(g_err_addr, dev, g_moba_device_error, &p);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(device error word)");
+  g->err = static_cast<int*>(p);
   return MOBA_OK;
 }
 
@@ -513,7 +531,7 @@ constexpr size_t kNoAllocMaxKbarElems = (size_t)1 << 21;  // hi + lo: 2 x 2^21 b
 static __device__ __align__(256) __nv_bfloat16 g_gate_scratch[2 * kNoAllocMaxKbarElems];
 
 namespace {
-__nv_bfloat16* g_gate_scratch_ptr[kMaxDevices] = {};
+SymbolAddress g_gate_scratch_addr;
 
 // Device address of g_gate_scratch on the current device, looked up once per device (the
 // host-side name of the array is only a stand-in, never a device address).
@@ -522,13 +540,10 @@ moba_status gate_scratch(__nv_bfloat16** out) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(MOBA_ERR_DEVICE, "device ordinal %d out of range", dev);
-  if (!g_gate_scratch_ptr[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_gate_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(gate scratch)");
-    g_gate_scratch_ptr[dev] = static_cast<__nv_bfloat16*>(ptr);
-  }
-  *out = g_gate_scratch_ptr[dev];
+  void* ptr = nullptr;
+  e = symbol_address(g_gate_scratch_addr, dev, g_gate_scratch, &ptr);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(gate scratch)");
+  *out = static_cast<__nv_bfloat16*>(ptr);
   return MOBA_OK;
 }
 }  // namespace

@@ -160,7 +160,9 @@ MOBA_API moba_status moba_attn_self_merge(const moba_params* p, const void* Q, c
  *    exceed MOBA_NOALLOC_MAX_KBAR_ELEMS (2^21; a 1M-token sequence with 8 KV heads of
  *    dimension 128 at block size 2048 needs 2^19); larger problems get MOBA_ERR_UNSUPPORTED.
  *  - The first call on each device looks up the array's device address (a CUDA runtime
- *    query, no allocation); make that first call before any stream capture begins.
+ *    query, no allocation; concurrent first calls from several host threads are safe); make
+ *    that first call before any stream capture begins.  The looked-up address belongs to the
+ *    device's primary context and is not valid after cudaDeviceReset on that device.
  *  - All calls share the one array and it keeps the last call's contents; every element a
  *    call reads is written earlier in the same call, so nothing needs clearing.  Calls
  *    whose kernels overlap on the GPU (other streams, other host threads) race on it and
