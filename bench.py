@@ -6,16 +6,24 @@ synthetic inputs already resident in HBM.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
 
+Besides the headline workload (1M tokens by default) the line carries
+  * ``configs``: the other long-context workloads (128K GQA, packed varlen) timed the
+    same way, with the attention's fraction of the measured bf16 peaks;
+  * ``dense_causal``: dense causal attention on the same GPU (torch SDPA, outside the
+    MoBA timed region) at the headline workload and at 32K MHA, and the library's own
+    full mode (top_k >= number of blocks) at 32K MHA;
+  * ``e2e``: the public host-buffer call with its host<->device copies timed;
+  * ``cpu_baseline``: the fp64 oracle on the host cores on a bounded row sample.
+
 Under torchrun (N > 1) every rank runs its own independent replica of the workload
 (the path has no cross-GPU exchange: problems shard by sequence and KV-head group),
-so scaling is weak; the timed region is bracketed by barriers and its length is the
+so scaling is weak; every timed region is bracketed by barriers and its length is the
 maximum over ranks.
 """
 from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -32,6 +40,9 @@ import synth  # noqa: E402
 
 METRIC = "MoBA fwd effective TFLOP/s & tokens/s at 1M ctx; % of B200 BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+STAGES = ("pool", "gate", "route", "past", "own")
+# the long-context workloads timed beside the headline one
+SIDE_CONFIGS = ("gqa128k", "varlen")
 
 
 def load_peaks():
@@ -55,6 +66,14 @@ def workload_desc(w: synth.Workload) -> str:
         ", ".join(extra))
 
 
+def config_dict(w: synth.Workload, world: int) -> dict:
+    """The workload description both arms print (same keys, same values)."""
+    q_gb = w.total_tokens * w.num_q_heads * w.head_dim * 2 / 1e9
+    return {"workload": workload_desc(w), "seq_len": w.max_seqlen, "global_batch": w.num_seqs * world,
+            "total_tokens_per_gpu": w.total_tokens, "parallelism": "replicas%d" % world,
+            "l2": "inputs larger than L2 (Q alone %.1f GB)" % q_gb}
+
+
 def flop_counts(w: synth.Workload, routed_rows: int) -> dict:
     """Algorithmic FLOPs of one pass: attention over unmasked attended keys, and the gate."""
     D, hq, bs = w.head_dim, w.num_q_heads, w.block_size
@@ -68,6 +87,11 @@ def flop_counts(w: synth.Workload, routed_rows: int) -> dict:
     own = 4 * D * hq * self_keys
     gate = 2 * D * hq * gate_dots
     return {"past": past, "own": own, "gate": gate, "attn": past + own}
+
+
+def dense_causal_flops(w: synth.Workload) -> int:
+    """4 D Hq sum_s S_s (S_s + 1) / 2: QK^T and PV over every causal key."""
+    return int(sum(4 * w.head_dim * w.num_q_heads * L * (L + 1) // 2 for L in w.seqlens))
 
 
 class ClockSampler:
@@ -207,6 +231,192 @@ def oracle_rows_per_second(w: synth.Workload, K: np.ndarray, V: np.ndarray, budg
 
 
 # --------------------------------------------------------------------------- our arm
+class MobaPass:
+    """Device buffers of one workload and one forward pass through the five C-ABI stages."""
+
+    def __init__(self, w: synth.Workload, dev, host=None, top_k: int | None = None):
+        import torch
+        import block_sparse_attention_gate_b200 as mb
+        self.mb = mb
+        self.w = w
+        self.dev = dev
+        if host is None:
+            host = make_host_inputs(w, pinned=False)
+        self.Q = host["q"].to(dev)
+        self.K = host["k"].to(dev)
+        self.V = host["v"].to(dev)
+        k = w.top_k if top_k is None else top_k
+        self.top_k = k
+        self.p = mb.MobaParams(w.cu_seqlens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, k)
+        self.ws = mb.alloc_workspace(self.p, dev)
+        T, hq, _ = self.Q.shape
+        self.kbar = torch.empty(self.p.kbar_elems, dtype=torch.float32, device=dev)
+        self.sel = torch.empty((T, hq, k), dtype=torch.int32, device=dev)
+        self.O = torch.empty_like(self.Q)
+        self.LSE = torch.empty((T, hq), dtype=torch.float32, device=dev)
+
+    def step(self, stream, ev=None):
+        mb, p = self.mb, self.p
+        if ev is not None:
+            ev[0].record(stream)
+        mb.moba_pool_keys(p, self.K, self.kbar, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        mb.moba_gate_topk(p, self.Q, self.kbar, self.sel, self.ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        mb.moba_route(p, self.sel, self.ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        mb.moba_attn_past(p, self.Q, self.K, self.V, self.ws, stream)
+        if ev is not None:
+            ev[4].record(stream)
+        mb.moba_attn_self_merge(p, self.Q, self.K, self.V, self.sel, self.ws, self.O, self.LSE, stream)
+        if ev is not None:
+            ev[5].record(stream)
+
+    def routed_rows(self) -> int:
+        if self.top_k < 2:
+            return 0
+        return int((self.sel[:, :, 1:] >= 0).sum().item())
+
+
+def time_pass(mp: MobaPass, steps: int, warmup: int, dist, clocks=None) -> dict:
+    """W untimed passes, then K passes timed by CUDA events on the launching stream (per
+    stage, between barriers and device synchronisations); max over ranks."""
+    import torch
+    dev = mp.dev
+    stream = torch.cuda.current_stream(dev)
+    warm = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for _ in range(warmup):
+        mp.step(stream, warm)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    if clocks is not None:
+        clocks.start()
+    torch.cuda.synchronize(dev)
+    for i in range(steps):
+        mp.step(stream, evs[i])
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop() if clocks is not None else None
+    total_ms = evs[0][0].elapsed_time(evs[-1][5])
+    stage_ms = {s: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / steps for j, s in enumerate(STAGES)}
+    return {"total_ms": max_over_ranks(total_ms, dist, dev), "stage_ms": stage_ms, "clocks": clk}
+
+
+def attn_fractions(fl: dict, stage_ms: dict, peaks: dict) -> dict:
+    attn_s = (stage_ms["past"] + stage_ms["own"]) / 1e3
+    attn_tf = fl["attn"] / attn_s / 1e12 if attn_s > 0 else 0.0
+    past_tf = fl["past"] / (stage_ms["past"] / 1e3) / 1e12 if stage_ms["past"] > 0 else 0.0
+    own_tf = fl["own"] / (stage_ms["own"] / 1e3) / 1e12 if stage_ms["own"] > 0 else 0.0
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    return {"attn_eff_tflops": attn_tf, "attn_frac_of_burst": attn_tf / burst,
+            "attn_frac_of_sustained": attn_tf / sus, "past_tflops": past_tf, "own_tflops": own_tf}
+
+
+def time_side_config(name: str, dev, dist, peaks: dict, steps: int = 3, warmup: int = 3) -> dict:
+    """One of the other long-context workloads, timed like the headline one."""
+    import torch
+    w = synth.CONFIGS[name]
+    mp = MobaPass(w, dev)
+    t = time_pass(mp, steps, warmup, dist)
+    routed = mp.routed_rows()
+    fl = flop_counts(w, routed)
+    ms = t["total_ms"] / steps
+    out = {"workload": workload_desc(w), "steps": steps, "warmup": warmup, "ms_per_step": ms,
+           "tokens_per_s": w.total_tokens / (ms / 1e3),
+           "eff_tflops": (fl["attn"] + fl["gate"]) / (ms / 1e3) / 1e12,
+           "stage_ms": t["stage_ms"], "routed_rows": routed, "flops": fl}
+    out.update(attn_fractions(fl, t["stage_ms"], peaks))
+    del mp
+    torch.cuda.empty_cache()
+    return out
+
+
+def sdpa_dense_causal_ms(Q, K, V, heads_per_call: int, reps: int = 1):
+    """Dense causal attention (torch SDPA, cuDNN backend if it accepts the call, else flash,
+    else memory-efficient) over [T, H, D] tensors of one sequence.  The inputs are first
+    laid out as contiguous [1, H, T, D] with K and V repeated over each GQA group (outside
+    the timed region); the calls then run over groups of query heads so that no tensor of
+    a call exceeds 2^31 elements.  Returns (ms per whole pass, backend name)."""
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    T, hq, D = Q.shape
+    G = hq // K.shape[1]
+    hpc = max(G, heads_per_call - heads_per_call % G)
+    q_all = Q.permute(1, 0, 2).contiguous().unsqueeze(0)
+    k_all = K.repeat_interleave(G, dim=1).permute(1, 0, 2).contiguous().unsqueeze(0)
+    v_all = V.repeat_interleave(G, dim=1).permute(1, 0, 2).contiguous().unsqueeze(0)
+    calls = [(q_all[:, h0:h0 + hpc], k_all[:, h0:h0 + hpc], v_all[:, h0:h0 + hpc]) for h0 in range(0, hq, hpc)]
+
+    def run_all(backend):
+        with sdpa_kernel([backend]):
+            for q, k, v in calls:
+                F.scaled_dot_product_attention(q, k, v, is_causal=True)
+
+    result = (None, "no SDPA backend accepted the call")
+    for backend, name in ((SDPBackend.CUDNN_ATTENTION, "cudnn"), (SDPBackend.FLASH_ATTENTION, "flash"),
+                          (SDPBackend.EFFICIENT_ATTENTION, "efficient")):
+        try:
+            run_all(backend)  # warm-up (plan build) on the same shapes
+            torch.cuda.synchronize()
+        except RuntimeError:
+            continue
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            run_all(backend)
+        b.record()
+        torch.cuda.synchronize()
+        result = (a.elapsed_time(b) / reps, name)
+        break
+    del calls, q_all, k_all, v_all
+    torch.cuda.empty_cache()
+    return result
+
+
+def dense_comparators(mp_main: MobaPass, main_ms: float, dev, dist) -> dict:
+    """Dense causal attention on the same GPU, outside the MoBA timed region."""
+    import torch
+    res = {}
+    w = mp_main.w
+    if w.num_seqs == 1:
+        ms, backend = sdpa_dense_causal_ms(mp_main.Q, mp_main.K, mp_main.V, heads_per_call=4)
+        ms = max_over_ranks(ms if ms is not None else -1.0, dist, dev)
+        fl = dense_causal_flops(w)
+        res[w.name] = {"impl": "torch SDPA dense causal (%s), heads in groups of 4" % backend,
+                       "ms": ms, "flops": fl, "tflops": fl / (ms / 1e3) / 1e12 if ms and ms > 0 else None,
+                       "moba_ms": main_ms, "moba_speedup": ms / main_ms if ms and ms > 0 else None}
+    # 32K MHA: SDPA, the library in its full mode (top_k = 16 = number of blocks) and MoBA top_k 3
+    w32 = synth.CONFIGS["mha32k"]
+    host = make_host_inputs(w32, pinned=False)
+    full = MobaPass(w32, dev, host=host, top_k=16)
+    t_full = time_pass(full, 5, 3, dist)
+    ms_sdpa, backend = sdpa_dense_causal_ms(full.Q, full.K, full.V, heads_per_call=32, reps=5)
+    ms_sdpa = max_over_ranks(ms_sdpa if ms_sdpa is not None else -1.0, dist, dev)
+    del full
+    moba = MobaPass(w32, dev, host=host)
+    t_moba = time_pass(moba, 5, 3, dist)
+    del moba
+    torch.cuda.empty_cache()
+    fl = dense_causal_flops(w32)
+    full_ms = t_full["total_ms"] / 5
+    moba_ms = t_moba["total_ms"] / 5
+    res["mha32k"] = {"sdpa_impl": "torch SDPA dense causal (%s)" % backend, "sdpa_ms": ms_sdpa,
+                     "sdpa_tflops": fl / (ms_sdpa / 1e3) / 1e12 if ms_sdpa > 0 else None,
+                     "library_full_ms": full_ms, "library_full_tflops": fl / (full_ms / 1e3) / 1e12,
+                     "library_full_stage_ms": t_full["stage_ms"], "flops": fl,
+                     "moba_top3_ms": moba_ms, "moba_speedup_vs_sdpa": ms_sdpa / moba_ms if ms_sdpa > 0 else None,
+                     "moba_speedup_vs_library_full": full_ms / moba_ms}
+    return res
+
+
 def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | None:
     import torch
     import block_sparse_attention_gate_b200 as mb
@@ -215,66 +425,26 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     host = make_host_inputs(w, pinned=True, nthreads=max(1, (os.cpu_count() or 1) // world))
-    Q = host["q"].to(dev, non_blocking=True)
-    K = host["k"].to(dev, non_blocking=True)
-    V = host["v"].to(dev, non_blocking=True)
-    p = mb.MobaParams(w.cu_seqlens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
-                      w.top_k)
-    ws = mb.alloc_workspace(p, dev)
-    T, hq, D = Q.shape
-    kbar = torch.empty(p.kbar_elems, dtype=torch.float32, device=dev)
-    sel = torch.empty((T, hq, w.top_k), dtype=torch.int32, device=dev)
-    O = torch.empty_like(Q)
-    LSE = torch.empty((T, hq), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    stages = ("pool", "gate", "route", "past", "own")
-
-    def step(ev):
-        ev[0].record(stream)
-        mb.moba_pool_keys(p, K, kbar, stream)
-        ev[1].record(stream)
-        mb.moba_gate_topk(p, Q, kbar, sel, ws, stream)
-        ev[2].record(stream)
-        mb.moba_route(p, sel, ws, stream)
-        ev[3].record(stream)
-        mb.moba_attn_past(p, Q, K, V, ws, stream)
-        ev[4].record(stream)
-        mb.moba_attn_self_merge(p, Q, K, V, sel, ws, O, LSE, stream)
-        ev[5].record(stream)
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    warm = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-    for _ in range(args.warmup):
-        step(warm)
-    torch.cuda.synchronize(dev)
-    if dist is not None:
-        dist.barrier()
+    mp = MobaPass(w, dev, host=host)
+    peaks, peak_kind = load_peaks()
     clocks = ClockSampler(local)
-    clocks.start()
-    torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        step(evs[i])
-    torch.cuda.synchronize(dev)
-    if dist is not None:
-        dist.barrier()
-    clk = clocks.stop()
-    total_ms = evs[0][0].elapsed_time(evs[-1][5])
-    stage_ms = {s: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j, s in enumerate(stages)}
-    t_max = max_over_ranks(total_ms, dist, dev)
-    routed = int((sel[:, :, 1:] >= 0).sum().item()) if w.top_k > 1 else 0
-    # sel slot >= 1 is valid exactly when it names a past block; verify the count from the rows
+    t = time_pass(mp, args.steps, args.warmup, dist, clocks)
+    stage_ms, clk = t["stage_ms"], t["clocks"]
+    t_max = t["total_ms"]
+    routed = mp.routed_rows()
     fl = flop_counts(w, routed)
     ms_step = t_max / args.steps
+    T = w.total_tokens
     tokens_per_s = job_throughput(T, world, args.steps, t_max)
 
     # ----- end to end through the public call with host buffers (pinned), copies timed
     e2e = None
     if not args.no_e2e:
         # the public host-buffer call: per-KV-group slices copied and computed over 3 streams
-        O_host = torch.empty(O.shape, dtype=torch.bfloat16, pin_memory=True)
-        L_host = torch.empty(LSE.shape, dtype=torch.float32, pin_memory=True)
+        O_host = torch.empty(mp.O.shape, dtype=torch.bfloat16, pin_memory=True)
+        L_host = torch.empty(mp.LSE.shape, dtype=torch.float32, pin_memory=True)
         streams = [torch.cuda.Stream(dev) for _ in range(3)]
-        staging = torch.empty(max(mb.moba_host_staging_size(p, len(streams)), 256), dtype=torch.uint8,
+        staging = torch.empty(max(mb.moba_host_staging_size(mp.p, len(streams)), 256), dtype=torch.uint8,
                               device=dev)
         n_e2e = max(1, min(args.steps, 3))
         main_stream = torch.cuda.current_stream(dev)
@@ -285,7 +455,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
             for s_ in streams:
                 s_.wait_event(a)
             for _ in range(n):
-                mb.moba_fwd_host(p, host["q"], host["k"], host["v"], O_host, L_host, staging, streams)
+                mb.moba_fwd_host(mp.p, host["q"], host["k"], host["v"], O_host, L_host, staging, streams)
             for s_ in streams:
                 ev = torch.cuda.Event()
                 ev.record(s_)
@@ -299,16 +469,16 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
             dist.barrier()
         e_ms = max_over_ranks(e2e_run(n_e2e), dist, dev)
         h2d = sum(host[x].numel() * 2 for x in ("q", "k", "v"))
-        d2h = O.numel() * 2 + LSE.numel() * 4
+        d2h = mp.O.numel() * 2 + mp.LSE.numel() * 4
         e2e = {"value": job_throughput(T, world, n_e2e, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+        del staging, streams
+        torch.cuda.empty_cache()
 
     traffic, traffic_note = past_kernel_traffic(routed)
-    peaks, peak_kind = load_peaks()
     peak_tf = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     past_s = stage_ms["past"] / 1e3
     achieved = fl["past"] / past_s / 1e12 if past_s > 0 else 0.0
-    attn_s = (stage_ms["past"] + stage_ms["own"]) / 1e3
     eff_tf = (fl["attn"] + fl["gate"]) / (ms_step / 1e3) / 1e12
     res = {
         "metric": METRIC,
@@ -323,11 +493,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded splitmix64/Box-Muller normals, RoPE, planted relevance per recipe)",
-        "config": {"workload": workload_desc(w), "seq_len": w.max_seqlen, "global_batch": w.num_seqs * world,
-                   "total_tokens_per_gpu": T, "parallelism": "replicas%d" % world,
-                   "l2": "inputs larger than L2 (Q alone %.1f GB)" % (Q.numel() * 2 / 1e9)},
+        "config": config_dict(w, world),
         "eff_tflops": eff_tf,
-        "attn_eff_tflops": fl["attn"] / attn_s / 1e12 if attn_s > 0 else 0.0,
         "pct_bf16_peak": 100.0 * eff_tf / peak_tf,
         "stage_ms": stage_ms,
         "flops": fl,
@@ -337,9 +504,16 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
                      "peak_kind": "%s bf16 sustained (kernel timed inside a long step)" % peak_kind,
                      "traffic": traffic, "traffic_note": traffic_note},
         "clocks": clk,
-        "gpu_launches": mb.moba_launches_per_forward(p) * args.steps,
+        "gpu_launches": mb.moba_launches_per_forward(mp.p) * args.steps,
         "e2e": e2e,
     }
+    res.update(attn_fractions(fl, stage_ms, peaks))
+    res["peaks"] = {"bf16_burst": peaks.get("bf16_tflops"), "bf16_sustained": peak_tf, "kind": peak_kind}
+    if not args.no_side:
+        res["configs"] = {name: time_side_config(name, dev, dist, peaks) for name in SIDE_CONFIGS
+                          if name != w.name}
+    if not args.no_dense:
+        res["dense_causal"] = dense_comparators(mp, ms_step, dev, dist)
     if rank == 0 and world == 1 and not args.no_cpu:
         Kh = host["k"].view(torch.int16).numpy().view(np.uint16)
         Vh = host["v"].view(torch.int16).numpy().view(np.uint16)
@@ -351,31 +525,39 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
     return res
 
 
-def run_reference(args, w: synth.Workload, rank: int) -> dict | None:
-    """The oracle (fp64 CPU, all host cores) on a bounded sample of the same workload."""
+def run_reference(args, w: synth.Workload, rank: int, world: int) -> dict | None:
+    """The oracle (fp64 CPU, all host cores) on a bounded sample of the same workload.
+
+    Each step is one bounded sample (about --ref-seconds of oracle rows plus one pooling
+    pass over all keys); ``ms_per_step`` is that measured step time, and ``value`` the
+    throughput it implies for the whole pass (tokens/s, per-row time extrapolated to every
+    row).  The extrapolated time of one whole pass is reported separately."""
     if rank != 0:
         return None
     Kh = w.fill("k")
     Vh = w.fill("v")
-    vals, rows_all, secs_all = [], 0, 0.0
+    vals, rows_all, secs_all, step_s = [], 0, 0.0, []
     for i in range(args.warmup + args.steps):
-        tps, nrows, secs, thr, pool_s = oracle_rows_per_second(
-            w, Kh, Vh, args.ref_seconds, seed=i)
+        t0 = time.perf_counter()
+        tps, nrows, secs, thr, pool_s = oracle_rows_per_second(w, Kh, Vh, args.ref_seconds, seed=i)
+        dt = time.perf_counter() - t0
         if i >= args.warmup:
             vals.append(tps)
             rows_all += nrows
             secs_all += secs
+            step_s.append(dt)
     v = statistics.mean(vals)
     T = w.total_tokens
     return {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * T / v,
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(step_s),
+        "ms_per_full_pass_extrapolated": 1e3 * T / v,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded)",
-        "config": {"workload": workload_desc(w), "seq_len": w.max_seqlen, "global_batch": w.num_seqs},
+        "data": "synthetic (seeded splitmix64/Box-Muller normals, RoPE, planted relevance per recipe)",
+        "config": config_dict(w, world),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
-                         "sample": "%d random query rows over %d steps (%.1f s) plus pooling, "
-                                   "extrapolated to all rows" % (rows_all, args.steps, secs_all)},
+                         "sample": "%d random query rows over %d steps (%.1f s of rows) plus one pooling "
+                                   "pass per step, extrapolated to all rows" % (rows_all, args.steps, secs_all)},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -389,14 +571,16 @@ def main(argv=None):
     ap.add_argument("--config", default="prefill1m", choices=sorted(synth.CONFIGS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-side", action="store_true", help="skip the other long-context workloads")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense causal comparators")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--ref-seconds", type=float, default=8.0)
+    ap.add_argument("--ref-seconds", type=float, default=4.0)
     args = ap.parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     w = synth.CONFIGS[args.config]
     if args.impl == "reference":
-        res = run_reference(args, w, rank)
+        res = run_reference(args, w, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
         return 0

@@ -73,3 +73,24 @@ def test_reference_arm_prints_its_line():
     line = json.loads(out.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_dense_causal_flops_closed_form():
+    # two sequences of 3 and 5 tokens, D 8, 2 heads: 4 * D * H * (1+2+3 + 1+2+3+4+5)
+    w = synth.Workload("d", [3, 5], 2, 1, 8, 128, 3, seed=1)
+    assert bench.dense_causal_flops(w) == 4 * 8 * 2 * (6 + 15)
+
+
+def test_reference_arm_reports_its_measured_step_and_the_same_config():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--config", "tiny", "--steps", "2", "--warmup", "1", "--ref-seconds", "0.3"],
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    # the same workload description as the GPU arm prints
+    assert line["config"] == bench.config_dict(synth.CONFIGS["tiny"], 1)
+    # a step is one bounded sample: its measured length, not the extrapolated full pass
+    assert 300.0 <= line["ms_per_step"] < 60_000.0
+    assert line["ms_per_full_pass_extrapolated"] == pytest.approx(
+        1e3 * synth.CONFIGS["tiny"].total_tokens / line["value"])
+    assert line["cpu_baseline"]["value"] == line["value"] == line["e2e"]["value"]
