@@ -6,11 +6,12 @@ Parity rule (MoBA prefill, bf16 inputs, fp32 accumulation):
     unchosen gate score) exceeds 1e-3 * max |score| over its candidates;
   * on rows whose selection matches: O within max-abs 1e-2 and mean-abs 1e-3,
     LSE within 1e-3 (absolute).  O is a bf16 output, whose own resolution is coarser than
-    1e-2 for |O| >= 4 (half an ulp there is 2^-6), so an element may also differ by the
-    rounding of the output itself (half a bf16 ulp of the exact value) plus 2e-3 for the
-    fp32 accumulation, the bf16 probabilities and the fp16 partials:
-    |O_gpu - O| <= max(1e-2, ulp_bf16(|O|) / 2 + 2e-3).  The statistics count the
-    elements that the widened bound covers and the ones that needed it;
+    1e-2 for |O| >= 2 (an ulp there is 2^-6), so an element may also differ by one bf16
+    ulp of the exact value: |O_gpu - O| <= max(1e-2, ulp_bf16(|O|)).  The ulp budget:
+    the output's own rounding (half an ulp) plus the bf16 rounding of the probabilities in
+    the P V product (up to 2^-9 sum_j P_j |V_j|, up to half an ulp more when a few keys
+    dominate a row), the fp16 partials (2^-11) and the fp32 accumulation.  The statistics
+    count the elements that the widened bound covers and the ones that needed it;
   * rows whose selection may legitimately differ (gap under the threshold) are
     excluded from the O/LSE comparison and counted.
 """
@@ -27,8 +28,6 @@ O_MEAN_ABS = 1e-3
 LSE_ABS = 1e-3
 # Kbar: fp32 sums of at most 8192 bf16 values of magnitude below ~10; observed errors are ~1e-6
 KBAR_ABS = 1e-4
-# accumulation slack added to half an output ulp in the widened O bound
-O_ACC_SLACK = 2e-3
 
 
 def bf16_ulp(x: np.ndarray) -> np.ndarray:
@@ -101,7 +100,7 @@ def compare(gpu_sel, gpu_O, gpu_LSE, orc: dict) -> dict:
     bad_sel = int(np.sum(qualified & ~same))
     d_o = np.abs(gpu_O.astype(np.float64) - orc["O"])[same]
     d_l = np.abs(gpu_LSE.astype(np.float64) - orc["lse"])[same]
-    wide = 0.5 * bf16_ulp(orc["O"][same]) + O_ACC_SLACK
+    wide = bf16_ulp(orc["O"][same])
     tol_o = np.maximum(O_MAX_ABS, wide)
     return {
         "rows": int(same.size),
