@@ -26,7 +26,8 @@ EXPORTS = ("moba_kbar_elems", "moba_workspace_size", "moba_pool_keys", "moba_gat
            "moba_attn_fwd", "moba_fwd", "moba_route", "moba_attn_past", "moba_attn_self_merge",
            "moba_launches_per_forward", "moba_read_device_error", "moba_status_string",
            "moba_last_error", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait",
-           "moba_host_staging_size", "moba_fwd_host")
+           "moba_host_staging_size", "moba_fwd_host", "moba_attn_naive", "moba_decode_workspace_size",
+           "moba_decode_fwd", "moba_pool_last_block", "moba_bwd_workspace_size", "moba_attn_bwd")
 
 
 class MobaError(RuntimeError):
@@ -72,6 +73,18 @@ def load():
         lib.moba_route.argtypes = [P, vp, vp, sz, vp]
         lib.moba_attn_past.argtypes = [P, vp, vp, vp, vp, sz, vp]
         lib.moba_attn_self_merge.argtypes = [P, vp, vp, vp, vp, vp, sz, vp, vp, vp]
+        lib.moba_bwd_workspace_size.argtypes = [P]
+        lib.moba_bwd_workspace_size.restype = sz
+        lib.moba_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp, vp]
+        lib.moba_attn_bwd.restype = ctypes.c_int
+        lib.moba_decode_workspace_size.argtypes = [P]
+        lib.moba_decode_workspace_size.restype = sz
+        lib.moba_decode_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp]
+        lib.moba_decode_fwd.restype = ctypes.c_int
+        lib.moba_pool_last_block.argtypes = [P, vp, vp, vp]
+        lib.moba_pool_last_block.restype = ctypes.c_int
+        lib.moba_attn_naive.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
+        lib.moba_attn_naive.restype = ctypes.c_int
         lib.moba_gate_topk_noalloc.argtypes = [P, vp, vp, vp, vp]
         lib.moba_gate_topk_noalloc.restype = ctypes.c_int
         lib.moba_host_staging_size.argtypes = [P, ctypes.c_int]
@@ -202,6 +215,42 @@ def moba_attn_self_merge(p: MobaParams, Q, K, V, sel, workspace, O, LSE, stream=
     _check(load().moba_attn_self_merge(p.ref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(sel), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _ptr(O), _ptr(LSE),
                                        _stream(stream)))
+
+
+def moba_attn_naive(p: MobaParams, Q, K, V, sel, O, LSE, stream=None) -> None:
+    """Mask-based attention over every causal key with the selection as a block mask
+    (a baseline for moba_attn_fwd; same results up to rounding)."""
+    _check(load().moba_attn_naive(p.ref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(sel), _ptr(O), _ptr(LSE),
+                                  _stream(stream)))
+
+
+def moba_bwd_workspace_size(p: MobaParams) -> int:
+    return int(load().moba_bwd_workspace_size(p.ref()))
+
+
+def moba_attn_bwd(p: MobaParams, Q, K, V, O, LSE, dO, sel, workspace, dQ, dK, dV, stream=None) -> None:
+    """Gradients dQ [T,Hq,D], dK, dV [T,Hkv,D] (bf16) of MoBA attention for dO, with the
+    forward's selection held fixed."""
+    _check(load().moba_attn_bwd(p.ref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), _ptr(dO), _ptr(sel),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dQ),
+                                _ptr(dK), _ptr(dV), _stream(stream)))
+
+
+def moba_decode_workspace_size(p: MobaParams) -> int:
+    return int(load().moba_decode_workspace_size(p.ref()))
+
+
+def moba_decode_fwd(p: MobaParams, Q, K, V, Kbar, workspace, O, LSE, sel=None, stream=None) -> None:
+    """Gated decode: Q [num_seqs, Hq, D] (the newest token of each cached sequence) against
+    the caches K, V [T, Hkv, D] described by p; O [num_seqs, Hq, D], LSE [num_seqs, Hq]."""
+    _check(load().moba_decode_fwd(p.ref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kbar), _ptr(sel), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _ptr(O), _ptr(LSE),
+                                  _stream(stream)))
+
+
+def moba_pool_last_block(p: MobaParams, K, Kbar, stream=None) -> None:
+    """Re-pool each sequence's last block into Kbar (after appending to a KV cache)."""
+    _check(load().moba_pool_last_block(p.ref(), _ptr(K), _ptr(Kbar), _stream(stream)))
 
 
 def moba_gate_topk_noalloc(p: MobaParams, Q, Kbar, sel, stream=None) -> None:

@@ -331,6 +331,182 @@ moba_status moba_attn_self_merge(const moba_params* p, const void* Q, const void
   return attn_stages(g, Q, K, V, sel, w, O, LSE, (cudaStream_t)stream, 4);
 }
 
+moba_status moba_attn_naive(const moba_params* p, const void* Q, const void* K, const void* V,
+                            const int32_t* sel, void* O, float* LSE, void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(Q, "Q", true));
+  MOBA_TRY(check_ptr(K, "K", true));
+  MOBA_TRY(check_ptr(V, "V", true));
+  MOBA_TRY(check_ptr(sel, "sel", true));
+  MOBA_TRY(check_ptr(O, "O", true));
+  MOBA_TRY(check_ptr(LSE, "LSE", true));
+  MOBA_TRY(check_device(&g));
+  cudaError_t e = moba::launch_attn_naive(g, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+                                          (const __nv_bfloat16*)V, sel, (__nv_bfloat16*)O, LSE,
+                                          (cudaStream_t)stream);
+  return e == cudaSuccess ? MOBA_OK : cuda_fail(e, "mask-based attention launch");
+}
+
+}  // extern "C"
+
+namespace {
+// Decode needs every sequence to hold at least the new token.
+moba_status check_decode_lengths(const moba_params* p) {
+  if (p->cu_seqlens_host) {
+    for (int s = 0; s < p->num_seqs; ++s)
+      if (p->cu_seqlens_host[s + 1] - p->cu_seqlens_host[s] < 1)
+        return fail(MOBA_ERR_INVALID_ARG, "decode: sequence %d is empty (the cache must hold the new token)", s);
+  } else if (p->max_seqlen < 1) {
+    return fail(MOBA_ERR_INVALID_ARG, "decode: max_seqlen must be >= 1");
+  }
+  return MOBA_OK;
+}
+
+struct DecodeWork {
+  float* part_o;
+  float* part_lse;
+  int32_t* sel;
+  size_t bytes;
+};
+
+DecodeWork carve_decode(const moba::Geom& g, char* base) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* ptr = base ? base + off : nullptr;
+    off += align256(bytes);
+    return ptr;
+  };
+  const size_t units = (size_t)g.num_seqs * g.Hq * g.k;
+  DecodeWork w;
+  w.part_o = (float*)take(units * g.D * sizeof(float));
+  w.part_lse = (float*)take(units * sizeof(float));
+  w.sel = (int32_t*)take(units * sizeof(int32_t));
+  w.bytes = off;
+  return w;
+}
+}  // namespace
+
+extern "C" {
+
+}  // extern "C"
+
+namespace {
+// Backward workspace: the routing arrays (as the forward's), Dp, fp32 dQ partials.
+struct BwdWork {
+  moba::Work route;
+  float* Dp;
+  float* dq_part;
+  size_t bytes;
+};
+
+BwdWork carve_bwd(const moba::Geom& g, char* base) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* ptr = base ? base + off : nullptr;
+    off += align256(bytes);
+    return ptr;
+  };
+  BwdWork w;
+  moba::Work x{};
+  x.counts = (int32_t*)take(sizeof(int32_t) * (size_t)g.nbk);
+  x.cursors = (int32_t*)take(sizeof(int32_t) * (size_t)g.nbk);
+  x.tile_off = (int32_t*)take(sizeof(int32_t) * (size_t)(g.nbk + 1));
+  x.tile_bucket = (int32_t*)take(sizeof(int32_t) * (size_t)moba::past_tiles(g));
+  x.rows = (int32_t*)take(sizeof(int32_t) * (size_t)moba::past_tiles(g) * moba::kPastTileRows);
+  w.route = x;
+  w.Dp = (float*)take(sizeof(float) * (size_t)g.T * g.Hq);
+  w.dq_part = (float*)take(sizeof(float) * (size_t)g.R * g.D);
+  w.bytes = off;
+  return w;
+}
+}  // namespace
+
+extern "C" {
+
+size_t moba_bwd_workspace_size(const moba_params* p) {
+  moba::Geom g;
+  if (make_geom(p, &g) != MOBA_OK) return 0;
+  return carve_bwd(g, nullptr).bytes;
+}
+
+moba_status moba_attn_bwd(const moba_params* p, const void* Q, const void* K, const void* V, const void* O,
+                          const float* LSE, const void* dO, const int32_t* sel, void* workspace,
+                          size_t workspace_bytes, void* dQ, void* dK, void* dV, void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(Q, "Q", true));
+  MOBA_TRY(check_ptr(K, "K", true));
+  MOBA_TRY(check_ptr(V, "V", true));
+  MOBA_TRY(check_ptr(O, "O", true));
+  MOBA_TRY(check_ptr(LSE, "LSE", true));
+  MOBA_TRY(check_ptr(dO, "dO", true));
+  MOBA_TRY(check_ptr(sel, "sel", true));
+  MOBA_TRY(check_ptr(dQ, "dQ", true));
+  MOBA_TRY(check_ptr(dK, "dK", true));
+  MOBA_TRY(check_ptr(dV, "dV", true));
+  const size_t need = carve_bwd(g, nullptr).bytes;
+  if (!workspace) return fail(MOBA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+  if (((uintptr_t)workspace) & 255) return fail(MOBA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (workspace_bytes < need) return fail(MOBA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, need);
+  MOBA_TRY(check_device(&g));
+  BwdWork w = carve_bwd(g, (char*)workspace);
+  cudaError_t e = moba::launch_attn_bwd(g, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
+                                        (const __nv_bfloat16*)O, LSE, (const __nv_bfloat16*)dO, sel, w.route, w.Dp,
+                                        w.dq_part, (__nv_bfloat16*)dQ, (__nv_bfloat16*)dK, (__nv_bfloat16*)dV,
+                                        (cudaStream_t)stream);
+  return e == cudaSuccess ? MOBA_OK : cuda_fail(e, "backward launch");
+}
+
+moba_status moba_pool_last_block(const moba_params* p, const void* K, float* Kbar, void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  if (g.T == 0 || g.MB == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(K, "K", true));
+  MOBA_TRY(check_ptr(Kbar, "Kbar", true));
+  MOBA_TRY(check_device(&g));
+  cudaError_t e = moba::launch_pool_last(g, (const __nv_bfloat16*)K, Kbar, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOBA_OK : cuda_fail(e, "pool (last block) launch");
+}
+
+size_t moba_decode_workspace_size(const moba_params* p) {
+  moba::Geom g;
+  if (make_geom(p, &g) != MOBA_OK) return 0;
+  return carve_decode(g, nullptr).bytes;
+}
+
+moba_status moba_decode_fwd(const moba_params* p, const void* Q, const void* K, const void* V, const float* Kbar,
+                            int32_t* sel, void* workspace, size_t workspace_bytes, void* O, float* LSE,
+                            void* stream) {
+  g_err[0] = 0;
+  moba::Geom g;
+  MOBA_TRY(make_geom(p, &g));
+  MOBA_TRY(check_decode_lengths(p));
+  if (g.T == 0) return MOBA_OK;
+  MOBA_TRY(check_ptr(Q, "Q", true));
+  MOBA_TRY(check_ptr(K, "K", true));
+  MOBA_TRY(check_ptr(V, "V", true));
+  MOBA_TRY(check_ptr(Kbar, "Kbar", true));
+  MOBA_TRY(check_ptr(sel, "sel", sel != nullptr));
+  MOBA_TRY(check_ptr(O, "O", true));
+  MOBA_TRY(check_ptr(LSE, "LSE", true));
+  const size_t need = carve_decode(g, nullptr).bytes;
+  if (!workspace) return fail(MOBA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+  if (((uintptr_t)workspace) & 255) return fail(MOBA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (workspace_bytes < need) return fail(MOBA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, need);
+  MOBA_TRY(check_device(&g));
+  DecodeWork w = carve_decode(g, (char*)workspace);
+  cudaError_t e = moba::launch_decode(g, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
+                                      Kbar, sel ? sel : w.sel, w.part_o, w.part_lse, (__nv_bfloat16*)O, LSE,
+                                      (cudaStream_t)stream);
+  return e == cudaSuccess ? MOBA_OK : cuda_fail(e, "decode launch");
+}
+
 int moba_launches_per_forward(const moba_params* p) {
   moba::Geom g;
   if (make_geom(p, &g) != MOBA_OK) return -1;

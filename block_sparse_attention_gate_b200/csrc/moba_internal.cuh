@@ -72,6 +72,13 @@ struct Work {
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, int heads, int D, int box_rows);
 cudaError_t launch_pool(const Geom& g, const __nv_bfloat16* K, float* Kbar, cudaStream_t st);
+// Pools only each sequence's last block (the one holding its newest token).
+cudaError_t launch_pool_last(const Geom& g, const __nv_bfloat16* K, float* Kbar, cudaStream_t st);
+// Gated decode: gate, split-KV attention over the selected blocks, merge.  part_o
+// [num_seqs * Hq * k, D] fp32 and part_lse [num_seqs * Hq * k] are scratch.
+cudaError_t launch_decode(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                          const float* Kbar, int32_t* sel, float* part_o, float* part_lse, __nv_bfloat16* O,
+                          float* LSE, cudaStream_t st);
 cudaError_t launch_gate(const Geom& g, const __nv_bfloat16* Q, const float* Kbar, int32_t* sel,
                         const Work& w, cudaStream_t st);
 cudaError_t launch_route(const Geom& g, const int32_t* sel, const Work& w, cudaStream_t st);
@@ -80,6 +87,17 @@ cudaError_t launch_attn_past(const Geom& g, const __nv_bfloat16* Q, const __nv_b
 cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                              const __nv_bfloat16* V, const int32_t* sel, const Work& w,
                              __nv_bfloat16* O, float* LSE, cudaStream_t st);
+// Mask-based form: every causal key scored, keys outside the selected blocks masked.
+cudaError_t launch_attn_naive(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                              const __nv_bfloat16* V, const int32_t* sel, __nv_bfloat16* O, float* LSE,
+                              cudaStream_t st);
+// Backward through the selected blocks (selection held fixed): Dp pre-pass, routing, dQ
+// partials of the routed slots, own block + final dQ, dK/dV.  Dp [T * Hq] and dq_part
+// [R, D] fp32 are scratch; w carries the routing arrays.
+cudaError_t launch_attn_bwd(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                            const __nv_bfloat16* O, const float* LSE, const __nv_bfloat16* dO, const int32_t* sel,
+                            const Work& w, float* Dp, float* dq_part, __nv_bfloat16* dQ, __nv_bfloat16* dK,
+                            __nv_bfloat16* dV, cudaStream_t st);
 // Number of kernel launches one forward pass enqueues (pool, gate, route, attention).
 int launches_per_forward(const Geom& g);
 

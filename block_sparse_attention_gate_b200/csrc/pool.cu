@@ -16,10 +16,13 @@ constexpr int kStripVec = 8;                            // 16-byte vectors per s
 constexpr int kStripCols = kStripVec * 8;               // 64 bf16 columns
 constexpr int kRowGroups = kPoolThreads / kStripVec;    // 32
 
+// last_only: grid.y is 1 and each sequence's last block (the one holding its newest token)
+// is pooled, for keeping Kbar current while a KV cache grows token by token.
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geom g, const __nv_bfloat16* __restrict__ K,
-                                                          float* __restrict__ Kbar) {
+                                                          float* __restrict__ Kbar, int last_only) {
   __shared__ float red[kRowGroups][kStripCols + 1];
-  const int strip = blockIdx.x, b = blockIdx.y, s = blockIdx.z;
+  const int strip = blockIdx.x, s = blockIdx.z;
+  const int b = last_only ? max(0, (seq_end(g, s) - seq_start(g, s) - 1) / g.bs) : (int)blockIdx.y;
   const int C = g.Hkv * g.D;
   const int32_t t0 = seq_start(g, s) + b * g.bs;
   const int32_t t1 = min(t0 + g.bs, seq_end(g, s));
@@ -70,7 +73,14 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geom g, const __nv_b
 cudaError_t launch_pool(const Geom& g, const __nv_bfloat16* K, float* Kbar, cudaStream_t st) {
   const int C = g.Hkv * g.D;  // a multiple of 64 (D is 64 or 128)
   dim3 grid(C / kStripCols, g.MB, g.num_seqs);
-  pool_kernel<<<grid, kPoolThreads, 0, st>>>(g, K, Kbar);
+  pool_kernel<<<grid, kPoolThreads, 0, st>>>(g, K, Kbar, 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool_last(const Geom& g, const __nv_bfloat16* K, float* Kbar, cudaStream_t st) {
+  const int C = g.Hkv * g.D;
+  dim3 grid(C / kStripCols, 1, g.num_seqs);
+  pool_kernel<<<grid, kPoolThreads, 0, st>>>(g, K, Kbar, 1);
   return cudaGetLastError();
 }
 

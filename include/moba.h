@@ -148,6 +148,76 @@ MOBA_API moba_status moba_attn_self_merge(const moba_params* p, const void* Q, c
                                           size_t workspace_bytes, void* O, float* LSE, void* stream);
 
 /*
+ * The mask-based form of the attention, as a baseline for the efficient path (README section
+ * "Implementation Details": moba_naive materialises the block-selection mask and runs masked
+ * attention; moba_efficient is the fast form).  Every causal key of the query's sequence is
+ * scored, and keys outside the row's selected blocks (from `sel`) get zero weight; the own
+ * block is causal.  Same O and LSE as moba_attn_fwd up to rounding, at the cost of dense
+ * causal attention (the tensor-core tiles of moba_attn_fwd's own-block stage, extended over
+ * the whole prefix).  Needs no workspace.
+ *   Q, K, V, sel, O, LSE: as for moba_attn_fwd.
+ */
+MOBA_API moba_status moba_attn_naive(const moba_params* p, const void* Q, const void* K, const void* V,
+                                     const int32_t* sel, void* O, float* LSE, void* stream);
+
+/*
+ * Backward pass through the selected blocks, for training (README bullet "Trainable Block
+ * Sparse Attention").  The gate has no parameters (README "Parameter-less Gating
+ * Mechanism"), so the top-k selection in `sel` is held fixed and the gradients are those
+ * of masked softmax attention under MoBA's mask (the selected blocks' keys, causal inside
+ * the own block): with P = exp(scale <q, k> - LSE), dP = <dO, v>, Dp = <dO, O> and
+ * dS = P (dP - Dp):  dQ = scale sum_j dS k_j,  dK = scale sum_p dS q_p,  dV = sum_p P dO_p
+ * (dK and dV summed over the query heads of each KV group).
+ *   Q, K, V, sel   the forward's inputs and selection (moba_gate_topk or moba_fwd).
+ *   O, LSE         the forward's outputs (O bf16 [T, Hq, D], LSE fp32 [T, Hq]).
+ *   dO             [T, Hq, D] bf16, the gradient of the loss with respect to O.
+ *   dQ             [T, Hq, D] bf16 out;  dK, dV  [T, Hkv, D] bf16 out.  Every element is
+ *                  written (keys that no query attends get 0).
+ *   workspace: >= moba_bwd_workspace_size(p) bytes, 256-byte aligned (routing arrays, Dp and
+ *   one fp32 dQ partial per routed (token, head, slot)).
+ * fp32 accumulation throughout; P and dS enter the tensor cores as bf16.
+ */
+MOBA_API size_t moba_bwd_workspace_size(const moba_params* p);
+MOBA_API moba_status moba_attn_bwd(const moba_params* p, const void* Q, const void* K, const void* V,
+                                   const void* O, const float* LSE, const void* dO, const int32_t* sel,
+                                   void* workspace, size_t workspace_bytes, void* dQ, void* dK, void* dV,
+                                   void* stream);
+
+/*
+ * Gated decode: one new query per sequence attends to that sequence's KV cache through the
+ * same gate as prefill (README: "Parameter-less Gating Mechanism"; README FAQ of issue #27:
+ * own block always taken, top_k-1 more from strictly earlier blocks; README FAQ of issue
+ * #30: the released decode path runs full attention instead, which this call does not).
+ * The new token is the LAST token of its sequence, at position p = len - 1 in block
+ * i = p / bs: its own (possibly partial) block is attended up to p, and the top_k - 1
+ * earlier blocks with the largest <q, Kbar[b]> are attended whole; the per-block results
+ * are merged by online softmax.  Results equal those of moba_fwd's row for that token.
+ *   p     the cache geometry: cu_seqlens over the cached tokens, which INCLUDE the new
+ *         token's key and value (every sequence holds >= 1 token, else MOBA_ERR_INVALID_ARG).
+ *   Q     [num_seqs, Hq, D] bf16: the new queries.
+ *   K, V  [T, Hkv, D] bf16: the caches.
+ *   Kbar  [num_seqs, MB, Hkv, D] fp32 pooled keys of the caches (moba_pool_keys once, then
+ *         moba_pool_last_block after each append keeps them current; only blocks before
+ *         each sequence's last block are read).
+ *   sel   [num_seqs, Hq, top_k] int32 out, as for moba_gate_topk; may be NULL.
+ *   workspace: >= moba_decode_workspace_size(p) bytes, 256-byte aligned.
+ *   O     [num_seqs, Hq, D] bf16 out;  LSE  [num_seqs, Hq] fp32 out.
+ */
+MOBA_API size_t moba_decode_workspace_size(const moba_params* p);
+MOBA_API moba_status moba_decode_fwd(const moba_params* p, const void* Q, const void* K, const void* V,
+                                     const float* Kbar, int32_t* sel, void* workspace, size_t workspace_bytes,
+                                     void* O, float* LSE, void* stream);
+
+/*
+ * Block mean-pooling of each sequence's LAST block only (the one holding its newest token),
+ * written into Kbar as moba_pool_keys would write it; every other block of Kbar is left
+ * untouched.  Reads at most block_size tokens per sequence: after appending tokens to a KV
+ * cache, this keeps Kbar equal to moba_pool_keys of the whole cache as long as each append
+ * stays within the sequence's current last block or opens the next one.
+ */
+MOBA_API moba_status moba_pool_last_block(const moba_params* p, const void* K, float* Kbar, void* stream);
+
+/*
  * moba_gate_topk without a workspace argument.  The MoBA pages have no counterpart: this is
  * an interface convenience, not part of the method.  Same inputs, outputs and results as
  * moba_gate_topk, for callers that cannot allocate device memory: code that enqueues work

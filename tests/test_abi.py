@@ -99,3 +99,42 @@ def test_host_staging_is_per_slot_group_sized():
     g = mb.MobaParams(None, G, 1, D, 2048, 3, num_seqs=1, max_seqlen=T)
     assert group_io + g.workspace_bytes <= one <= group_io + g.workspace_bytes + 8 * 256
     assert mb.moba_host_staging_size(p, 0) == 0
+
+
+def test_backward_and_decode_workspace_sizes():
+    # backward: routing arrays as in the forward, Dp (T*Hq fp32), one fp32 dQ partial per routed slot
+    T, hq, hkv, D, bs, k = 1 << 16, 32, 8, 128, 2048, 3
+    p = mb.MobaParams(None, hq, hkv, D, bs, k, num_seqs=1, max_seqlen=T)
+    R = T * hq * (k - 1)
+    bw = mb.moba_bwd_workspace_size(p)
+    assert R * D * 4 + T * hq * 4 + R * 4 <= bw <= R * D * 4 + T * hq * 4 + R * 4 + (R // 256 + 64) * 4 * 260 + 8 * 256
+    # decode: an fp32 partial O, its LSE and a selection slot per (sequence, head, slot)
+    q = mb.MobaParams(None, hq, hkv, D, bs, k, num_seqs=64, max_seqlen=T)
+    units = 64 * hq * k
+    assert mb.moba_decode_workspace_size(q) == (units * D * 4 + 255) // 256 * 256 + 2 * ((units * 4 + 255) // 256 * 256)
+
+
+def test_decode_rejects_empty_caches_before_any_cuda_call():
+    lib = mb.load()
+    arr = np.array([0, 5, 5, 9], dtype=np.int32)  # the second sequence is empty
+    c = mb._CParams()
+    c.num_seqs = 3
+    c.cu_seqlens_host = arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    c.cu_seqlens = 256
+    c.num_q_heads, c.num_kv_heads, c.head_dim, c.block_size, c.top_k = 2, 1, 64, 128, 3
+    rc = lib.moba_decode_fwd(ctypes.byref(c), 16, 16, 16, 16, None, 256, 1 << 20, 16, 16, None)
+    assert rc == 1 and b"empty" in lib.moba_last_error()
+    p = mb.MobaParams(None, 2, 1, 64, 128, 3, num_seqs=2, max_seqlen=0)
+    assert lib.moba_decode_fwd(p.ref(), 16, 16, 16, 16, None, 256, 1 << 20, 16, 16, None) == 1
+
+
+def test_backward_and_naive_check_arguments_before_any_cuda_call():
+    lib = mb.load()
+    p = mb.MobaParams(None, 2, 1, 64, 128, 3, num_seqs=1, max_seqlen=256)
+    ws = mb.moba_bwd_workspace_size(p)
+    # a NULL gradient, a misaligned output, a short workspace
+    assert lib.moba_attn_bwd(p.ref(), 16, 16, 16, 16, 16, None, 16, 256, ws, 16, 16, 16, None) == 1
+    assert lib.moba_attn_bwd(p.ref(), 16, 16, 16, 16, 16, 16, 16, 256, ws, 16, 18, 16, None) == 3
+    assert lib.moba_attn_bwd(p.ref(), 16, 16, 16, 16, 16, 16, 16, 256, ws - 1, 16, 16, 16, None) == 4
+    assert lib.moba_attn_naive(p.ref(), 16, 16, 16, None, 16, 16, None) == 1
+    assert lib.moba_pool_last_block(p.ref(), 18, 16, None) == 3
