@@ -266,15 +266,18 @@ __global__ void __launch_bounds__(kQThreads, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[qDQFull0 + t], 0, g.err));
     if (ok) {
       tc_fence_after();
-      // own mode: the row's past partials (slots naming an earlier block)
+      // own mode: the row's past partials.  The chosen past blocks fill slots 1..np of the
+      // row (the selection's padding is at the end), so partial q has the id row*(k-1) + q.
       int np = 0;
-      int64_t pe[kMaxTopK - 1];
+      const int64_t pbase = qrow >= 0 ? qrow * (g.k - 1) : 0;
       if constexpr (kOwn) {
         if (qrow >= 0) {
+          bool run = true;
 #pragma unroll
           for (int q = 0; q < kMaxTopK - 1; ++q) {
             const int32_t b = q + 1 < g.k ? __ldg(a.sel + qrow * g.k + q + 1) : -1;
-            if (b >= 0 && b < i_blk) pe[np++] = qrow * (g.k - 1) + q;
+            run = run && b >= 0 && b < i_blk;
+            np += run ? 1 : 0;
           }
         }
       }
@@ -288,7 +291,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         for (int x = 0; x < 32; ++x) v[x] = __uint_as_float(o[x]) * g.scale;
         if constexpr (kOwn) {
           for (int q = 0; q < np; ++q) {
-            const float4* src = reinterpret_cast<const float4*>(a.dq_part + pe[q] * D + c * 32);
+            const float4* src = reinterpret_cast<const float4*>(a.dq_part + (pbase + q) * D + c * 32);
 #pragma unroll
             for (int x = 0; x < 8; ++x) {
               const float4 f = __ldg(src + x);
@@ -418,6 +421,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 constexpr int kKVThreads = 288;  // warps 0-3 keys (TMEM lanes), 4-7 row gather, 8 TMA + MMA
 constexpr int kKeys = 128;       // keys per CTA (M)
 constexpr int kSub = 64;         // query rows per sub-tile (N of S^T)
+constexpr int kStages = 4;       // gathered sub-tiles in flight
 constexpr uint32_t kKColS = 0;     // S^T of buffer b at 64 b (P^T over its first 32 columns, dS^T over the next 32)
 constexpr uint32_t kKColDP = 128;  // dP^T of buffer b at 128 + 64 b
 constexpr uint32_t kKColDV = 256;  // dV, then dK at 256 + D
@@ -428,17 +432,17 @@ struct KVLayout {
   static constexpr int kSubT = kSub * D * 2;    // [64 x D]
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTile;
-  static constexpr int kQ0 = kV + kTile;        // two stages
-  static constexpr int kG0 = kQ0 + 2 * kSubT;   // two stages
-  static constexpr int kLse = kG0 + 2 * kSubT;  // [2][64] fp32
-  static constexpr int kDp = kLse + 2 * kSub * 4;
-  static constexpr int kBar = kDp + 2 * kSub * 4;
+  static constexpr int kQ0 = kV + kTile;              // kStages stages
+  static constexpr int kG0 = kQ0 + kStages * kSubT;   // kStages stages
+  static constexpr int kLse = kG0 + kStages * kSubT;  // [kStages][64] fp32 (natural-log LSE)
+  static constexpr int kDp = kLse + kStages * kSub * 4;
+  static constexpr int kBar = kDp + kStages * kSub * 4;
   static constexpr int kBytes = kBar + 256;
   static constexpr int kAlloc = kBytes + 1024 > 120 * 1024 ? kBytes + 1024 : 120 * 1024;  // one CTA per SM
 };
 
-enum KBar { kbKVFull = 0, kbStFull0, kbStFull1, kbStFree0, kbStFree1, kbSFull0, kbSFull1, kbPFull0, kbPFull1,
-            kbDone, kbNumBars };
+enum KBar { kbKVFull = 0, kbStFull0, kbStFree0 = kbStFull0 + kStages, kbSFull0 = kbStFree0 + kStages, kbSFull1,
+            kbPFull0, kbPFull1, kbDone, kbNumBars };
 
 // Rows of sub-tile n of a dK/dV CTA: the bucket's routed rows first, then the own block's
 // rows (per query head of the group, 64 tokens at a time, from the key tile onward).
@@ -485,9 +489,16 @@ __global__ void __launch_bounds__(kKVThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ------------------------------------------------------------- work item
+  // Blocks in ascending order, so the CTAs of early blocks (which later queries may choose,
+  // hence the larger buckets) start first; inside a block: sequence, KV head, key tile.
   const int per_blk = g.bs / kKeys;
-  const int b = blockIdx.x / per_blk, kt = blockIdx.x - b * per_blk;
-  const int s = blockIdx.y, gk = blockIdx.z;
+  int64_t idx = blockIdx.x;
+  const int kt = (int)(idx % per_blk);
+  idx /= per_blk;
+  const int gk = (int)(idx % g.Hkv);
+  idx /= g.Hkv;
+  const int s = (int)(idx % g.num_seqs);
+  const int b = (int)(idx / g.num_seqs);
   const int32_t ts = seq_start(g, s), te = seq_end(g, s);
   const int32_t blk0 = ts + b * g.bs;
   const int32_t key0 = blk0 + kt * kKeys;
@@ -515,9 +526,11 @@ __global__ void __launch_bounds__(kKVThreads, 1)
   }
   if (tid == 0) {
     mbar_init(&bars[kbKVFull], 1);
-    for (int q = 0; q < 2; ++q) {
-      mbar_init(&bars[kbStFull0 + q], 128);
+    for (int q = 0; q < kStages; ++q) {
+      mbar_init(&bars[kbStFull0 + q], 128);  // one (asynchronous) arrival per gather thread
       mbar_init(&bars[kbStFree0 + q], 1);
+    }
+    for (int q = 0; q < 2; ++q) {
       mbar_init(&bars[kbSFull0 + q], 1);
       mbar_init(&bars[kbPFull0 + q], kKeys);
     }
@@ -536,9 +549,9 @@ __global__ void __launch_bounds__(kKVThreads, 1)
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float c2 = g.scale_log2;
     for (int n = 0; n < N && ok; ++n) {
-      const int buf = n & 1;
+      const int buf = n & 1, st = n % kStages;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[kbSFull0 + buf], (n >> 1) & 1, g.err) &&
-                                       mbar_wait(&bars[kbStFull0 + buf], (n >> 1) & 1, g.err));
+                                       mbar_wait(&bars[kbStFull0 + st], (n / kStages) & 1, g.err));
       if (!ok) break;
       tc_fence_after();
       uint32_t sv[2][32], dv[2][32];
@@ -553,16 +566,17 @@ __global__ void __launch_bounds__(kKVThreads, 1)
       int own_sub = -1;
       if (n >= w.n_rsub) own_sub = (n - w.n_rsub) % w.n_osub_h;
       const int rmin = own_sub >= 0 ? k - own_sub * kSub : 0;  // first visible row
-      const float* lse = s_lse + buf * kSub;
-      const float* dpv = s_dp + buf * kSub;
+      // an empty row has Q = dO = 0 and LSE = Dp = 0: its P is 1 but dS and P dO vanish
+      const float* lse = s_lse + st * kSub;
+      const float* dpv = s_dp + st * kSub;
       uint32_t pp[32], pd[32];
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
           const int r = h2 * 32 + x;
-          float p0 = ex2(fmaf(__uint_as_float(sv[h2][x]), c2, -lse[r]));
-          float p1 = ex2(fmaf(__uint_as_float(sv[h2][x + 1]), c2, -lse[r + 1]));
+          float p0 = ex2(fmaf(__uint_as_float(sv[h2][x]), c2, lse[r] * -kLog2e));
+          float p1 = ex2(fmaf(__uint_as_float(sv[h2][x + 1]), c2, lse[r + 1] * -kLog2e));
           if (r < rmin) p0 = 0.f;
           if (r + 1 < rmin) p1 = 0.f;
           const float d0 = p0 * (__uint_as_float(dv[h2][x]) - dpv[r]);
@@ -607,27 +621,32 @@ __global__ void __launch_bounds__(kKVThreads, 1)
     }
   } else if (warp < 8) {
     // ========================================================= row gather (128 threads)
+    // Thread (r, which) copies row r of Q (which 0) or dO (which 1) of every sub-tile, and
+    // that row's LSE or Dp; the copies of kStages sub-tiles are in flight at once, each
+    // stage's barrier receiving the thread's arrival when its copies have landed.  The
+    // (token, head) row of each slot is looked up two sub-tiles ahead.
     const int p = tid - 128;
-    const int r = p >> 1, which = p & 1;  // row of the sub-tile; 0: Q, 1: dO
+    const int r = p >> 1, which = p & 1;
+    int own_sub;
+    int64_t q_a = N > 0 ? kv_row(g, a.rows, w, gk, 0, r, &own_sub) : -1;
+    int64_t q_b = N > 1 ? kv_row(g, a.rows, w, gk, 1, r, &own_sub) : -1;
     for (int n = 0; n < N && ok; ++n) {
-      const int st = n & 1, u = n >> 1;
+      const int st = n % kStages, u = n / kStages;
+      const int64_t qrow = q_a;
+      q_a = q_b;
+      q_b = n + 2 < N ? kv_row(g, a.rows, w, gk, n + 2, r, &own_sub) : -1;
       if (u > 0) ok = mbar_wait(&bars[kbStFree0 + st], (u - 1) & 1, g.err);
       if (!ok) break;
-      int own_sub;
-      const int64_t qrow = kv_row(g, a.rows, w, gk, n, r, &own_sub);
       const __nv_bfloat16* src = (which ? a.dO : a.Q) + (qrow >= 0 ? qrow * D : 0);
       const uint32_t nb = qrow >= 0 ? 16u : 0u;
       const uint32_t dstb = smem_u32(smem + (which ? L::kG0 : L::kQ0) + st * L::kSubT);
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) cp_async_16(dstb + sw128_offset(r, c, kSub), src + c * 8, nb);
-      if (which == 0) {
-        s_lse[st * kSub + r] = qrow >= 0 ? __ldg(a.LSE + qrow) * kLog2e : INFINITY;
-        s_dp[st * kSub + r] = qrow >= 0 ? __ldg(a.Dp + qrow) : 0.f;
-      }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(&bars[kbStFull0 + st]);
+      const float* sv = (which ? a.Dp : a.LSE) + (qrow >= 0 ? qrow : 0);
+      cp_async_4(smem_u32((which ? s_dp : s_lse) + st * kSub + r), sv, qrow >= 0 ? 4u : 0u);
+      cp_async_arrive_noinc(&bars[kbStFull0 + st]);
     }
+    cp_async_wait_all();  // nothing of this thread is in flight when the CTA ends
   } else {
     // ========================================================= TMA + MMA issuer (warp 8)
     if (lane == 0) {
@@ -647,45 +666,48 @@ __global__ void __launch_bounds__(kKVThreads, 1)
     const uint32_t sV = smem_u32(smem + L::kV);
     const uint32_t sQ0 = smem_u32(smem + L::kQ0);
     const uint32_t sG0 = smem_u32(smem + L::kG0);
-    auto issue_s = [&](int n) {  // S^T = K Q_n^T, dP^T = V dO_n^T into buffer n & 1
-      const int st = n & 1;
+    auto issue_s = [&](int n) {  // S^T = K Q_n^T, dP^T = V dO_n^T into TMEM buffer n & 1
+      const int st = n % kStages, buf = n & 1;
       const uint32_t qb = sQ0 + st * L::kSubT, gb = sG0 + st * L::kSubT;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t aoff = (kk >> 2) * (kKeys * 128) + (kk & 3) * 32;
         const uint32_t boff = (kk >> 2) * (kSub * 128) + (kk & 3) * 32;
-        mma_bf16_ss_warp(tmem + kKColS + st * kSub, sdesc_sw128(sK + aoff, 16, 1024), sdesc_sw128(qb + boff, 16, 1024),
-                         idS, kk > 0 ? 1u : 0u);
-        mma_bf16_ss_warp(tmem + kKColDP + st * kSub, sdesc_sw128(sV + aoff, 16, 1024),
+        mma_bf16_ss_warp(tmem + kKColS + buf * kSub, sdesc_sw128(sK + aoff, 16, 1024),
+                         sdesc_sw128(qb + boff, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        mma_bf16_ss_warp(tmem + kKColDP + buf * kSub, sdesc_sw128(sV + aoff, 16, 1024),
                          sdesc_sw128(gb + boff, 16, 1024), idS, kk > 0 ? 1u : 0u);
       }
-      mma_commit_warp(&bars[kbSFull0 + st]);
+      mma_commit_warp(&bars[kbSFull0 + buf]);
     };
     auto issue_acc = [&](int n) {  // dV += P^T dO_n, dK += dS^T Q_n
-      const int st = n & 1;
+      const int st = n % kStages, buf = n & 1;
       const uint32_t qb = sQ0 + st * L::kSubT, gb = sG0 + st * L::kSubT;
 #pragma unroll
       for (int kk = 0; kk < kSub / 16; ++kk) {
         const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-        mma_bf16_ts_warp(tmem + kKColDV, tmem + kKColS + st * kSub + kk * 8,
+        mma_bf16_ts_warp(tmem + kKColDV, tmem + kKColS + buf * kSub + kk * 8,
                          sdesc_sw128(gb + kk * 2048, kSub * 128, 1024), idG, acc);
-        mma_bf16_ts_warp(tmem + kKColDV + D, tmem + kKColS + st * kSub + 32 + kk * 8,
+        mma_bf16_ts_warp(tmem + kKColDV + D, tmem + kKColS + buf * kSub + 32 + kk * 8,
                          sdesc_sw128(qb + kk * 2048, kSub * 128, 1024), idG, acc);
       }
       mma_commit_warp(&bars[kbStFree0 + st]);
     };
+    // the gathered rows were written by cp.async (generic proxy): fence before the MMAs read them
     ok = mbar_wait_warp(&bars[kbKVFull], 0, g.err);
     if (ok && N > 0) {
       ok = mbar_wait_warp(&bars[kbStFull0], 0, g.err);
       if (ok) {
+        fence_proxy_async_smem();
         tc_fence_after();
         issue_s(0);
       }
     }
     for (int n = 0; n < N && ok; ++n) {
       if (n + 1 < N) {
-        ok = mbar_wait_warp(&bars[kbStFull0 + ((n + 1) & 1)], ((n + 1) >> 1) & 1, g.err);
+        ok = mbar_wait_warp(&bars[kbStFull0 + ((n + 1) % kStages)], ((n + 1) / kStages) & 1, g.err);
         if (!ok) break;
+        fence_proxy_async_smem();
         tc_fence_after();
         issue_s(n + 1);
       }
@@ -744,8 +766,8 @@ cudaError_t launch_bwd_d(const Geom& g, const BwdArgs& a, const __nv_bfloat16* K
     if ((e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
       return e;
-    const dim3 grid((unsigned)(g.MB * (g.bs / kKeys)), (unsigned)g.num_seqs, (unsigned)g.Hkv);
-    bwd_dkdv_kernel<D><<<grid, kKVThreads, smem, st>>>(tk128, tv128, a);
+    const int64_t nct = (int64_t)g.MB * g.num_seqs * g.Hkv * (g.bs / kKeys);
+    bwd_dkdv_kernel<D><<<(unsigned)nct, kKVThreads, smem, st>>>(tk128, tv128, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -90,6 +90,9 @@ struct AttnArgs {
   __nv_bfloat16* O;
   float* LSE;
   int own_head_pairs;  // own mode: tiles are heads (2p, 2p+1) of one group (else query tiles 2p, 2p+1)
+  int premerged;       // own mode: rows with two or more past partials have them folded in mo/mlse
+  const __half* mo;    // [T * Hq, D] folded partial of each such row
+  const float* mlse;   // [T * Hq] its LSE
 };
 
 template <int D>
@@ -228,6 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (row * (top_k - 1) + q).
   int np = 0;                 // own mode: past partials of this thread's row
   float pmax = -INFINITY;     // own mode: their largest LSE, log2 units
+  bool folded = false;        // own mode: the row's partials come folded (one partial in mo/mlse)
   if (kOwn && !kNaive && warp < 8) {
     const int t = warp >> 2, r = tid & (kRows - 1);
     if (r < ti[t].nrows) {
@@ -239,7 +243,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         run = run && b >= 0 && b < i_blk;
         np += run ? 1 : 0;
       }
-      for (int q = 0; q < np; ++q) pmax = fmaxf(pmax, __ldg(a.part_lse + qrow * (g.k - 1) + q) * kLog2e);
+      if (a.premerged && np >= 2) {
+        folded = true;
+        np = 1;
+        pmax = __ldg(a.mlse + qrow) * kLog2e;
+      } else {
+        for (int q = 0; q < np; ++q) pmax = fmaxf(pmax, __ldg(a.part_lse + qrow * (g.k - 1) + q) * kLog2e);
+      }
     }
   }
   // Past mode: the softmax threads look up their routed rows and start the Q gather before
@@ -335,8 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h2 = 0; h2 < 2; ++h2) {
           const int q = q0 + h2;
           const bool have = q < np;
-          w[h2] = have ? ex2(__ldg(a.part_lse + pbase + q) * kLog2e - m) : 0.f;
-          const uint4* src = reinterpret_cast<const uint4*>(a.part_o + (have ? pbase + q : 0) * D);
+          w[h2] = have ? ex2(__ldg(folded ? a.mlse + qrow : a.part_lse + pbase + q) * kLog2e - m) : 0.f;
+          const __half* srow = !have ? a.part_o : (folded ? a.mo + qrow * D : a.part_o + (pbase + q) * D);
+          const uint4* src = reinterpret_cast<const uint4*>(srow);
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) hv[h2][c] = have ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
         }
@@ -641,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, int kMode>
 cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                       const int32_t* sel, const Work& w, __nv_bfloat16* O, float* LSE, dim3 grid, int head_pairs,
-                      cudaStream_t st) {
+                      cudaStream_t st, int premerged = 0) {
   CUtensorMap tq, tk, tv;
   cudaError_t e = make_rows_map(&tk, K, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
@@ -653,7 +664,8 @@ cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16
   }
   e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
-  AttnArgs a{g, Q, sel, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, O, LSE, head_pairs};
+  AttnArgs a{g, Q, sel, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, O, LSE, head_pairs, premerged,
+             w.merged_o, w.merged_lse};
   const int smem = Layout<D>::kAlloc;
   e = cudaFuncSetAttribute(attn_tc_kernel<D, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -1020,7 +1032,8 @@ cudaError_t launch_past_persistent(const Geom& g, const __nv_bfloat16* K, const 
   if (e != cudaSuccess) return e;
   e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
-  AttnArgs a{g, Q, nullptr, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, nullptr, nullptr, 0};
+  AttnArgs a{g, Q, nullptr, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, nullptr, nullptr, 0, 0,
+             nullptr, nullptr};
   const int smem = PLayout<D>::kAlloc;
   e = cudaFuncSetAttribute(attn_past_persistent_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -1056,14 +1069,84 @@ dim3 own_grid(const Geom& g, int* head_pairs) {
 }
 }  // namespace
 
+namespace {
+// When a row can have more than two past partials, they are folded before the own-block
+// kernel runs: one warp per (token, head) row with two or more partials loads all of them
+// at once (a lane holds D/32 elements of each, so every partial row is one coalesced read),
+// merges them by online softmax (M = max LSE_q, w_q = e^(LSE_q - M), O = sum w_q O_q /
+// sum w_q, LSE = M + ln sum w_q) and writes the result to the row's entry of mo / mlse.
+// The own-block kernel then merges one partial per row: a single round trip instead of one
+// per two partials.  The partials themselves are left as they are.
+
+template <int D>
+__global__ void __launch_bounds__(256) premerge_kernel(Geom g, const int32_t* __restrict__ sel,
+                                                       const __half* __restrict__ part_o,
+                                                       const float* __restrict__ part_lse, __half* __restrict__ mo,
+                                                       float* __restrict__ mlse) {
+  constexpr int kDL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = (int64_t)g.T * g.Hq;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int km1 = g.k - 1;
+  for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows; row += nwarps) {
+    const int32_t t = (int32_t)(row / g.Hq);
+    const int s = find_seq(g, t);
+    const int i = (t - seq_start(g, s)) / g.bs;
+    // the row's past partials: the chosen past blocks fill the first np slots
+    int np = 0;
+    bool run = true;
+    for (int q = 0; q < km1; ++q) {
+      const int32_t b = __ldg(sel + row * g.k + 1 + q);
+      run = run && b >= 0 && b < i;
+      np += run ? 1 : 0;
+    }
+    if (np < 2) continue;
+    const int64_t base = row * km1;
+    float M = -INFINITY;
+    for (int q = 0; q < np; ++q) M = fmaxf(M, __ldg(part_lse + base + q));
+    float L = 0.f, acc[kDL];
+#pragma unroll
+    for (int x = 0; x < kDL; ++x) acc[x] = 0.f;
+#pragma unroll 4
+    for (int q = 0; q < np; ++q) {
+      const float w = __expf(__ldg(part_lse + base + q) - M);
+      L += w;
+      const __half2* src = reinterpret_cast<const __half2*>(part_o + (base + q) * D + lane * kDL);
+#pragma unroll
+      for (int x = 0; x < kDL / 2; ++x) {
+        const float2 f = __half22float2(src[x]);
+        acc[2 * x] = fmaf(w, f.x, acc[2 * x]);
+        acc[2 * x + 1] = fmaf(w, f.y, acc[2 * x + 1]);
+      }
+    }
+    const float inv = 1.f / L;
+    __half2* dst = reinterpret_cast<__half2*>(mo + row * D + lane * kDL);
+#pragma unroll
+    for (int x = 0; x < kDL / 2; ++x) dst[x] = __floats2half2_rn(acc[2 * x] * inv, acc[2 * x + 1] * inv);
+    if (lane == 0) mlse[row] = M + __logf(L);
+  }
+}
+}  // namespace
+
 cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                              const __nv_bfloat16* V, const int32_t* sel, const Work& w,
                              __nv_bfloat16* O, float* LSE, cudaStream_t st) {
   if (g.T == 0) return cudaSuccess;
   int head_pairs = 0;
   const dim3 grid = own_grid(g, &head_pairs);
-  if (g.D == 64) return launch_tc<64, kModeOwn>(g, Q, K, V, sel, w, O, LSE, grid, head_pairs, st);
-  return launch_tc<128, kModeOwn>(g, Q, K, V, sel, w, O, LSE, grid, head_pairs, st);
+  int premerged = 0;
+  if (premerge_used(g)) {
+    const int64_t rows = (int64_t)g.T * g.Hq;
+    const int64_t want = (rows + 7) / 8;
+    const unsigned blocks = (unsigned)(want < 148 * 64 ? want : 148 * 64);
+    if (g.D == 64) premerge_kernel<64><<<blocks, 256, 0, st>>>(g, sel, w.part_o, w.part_lse, w.merged_o, w.merged_lse);
+    else premerge_kernel<128><<<blocks, 256, 0, st>>>(g, sel, w.part_o, w.part_lse, w.merged_o, w.merged_lse);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    premerged = 1;
+  }
+  if (g.D == 64) return launch_tc<64, kModeOwn>(g, Q, K, V, sel, w, O, LSE, grid, head_pairs, st, premerged);
+  return launch_tc<128, kModeOwn>(g, Q, K, V, sel, w, O, LSE, grid, head_pairs, st, premerged);
 }
 
 cudaError_t launch_attn_naive(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
@@ -1079,8 +1162,9 @@ cudaError_t launch_attn_naive(const Geom& g, const __nv_bfloat16* Q, const __nv_
 
 int launches_per_forward(const Geom& g) {
   // pool + gate (Kbar split, scores/top-k) + (route count, scan, scatter + past attention
-  // when top_k > 1) + own block/merge
-  return 3 + (g.k > 1 ? 4 : 0) + 1;
+  // when top_k > 1) + (partial pre-merge when a row can have more than two partials) +
+  // own block/merge
+  return 3 + (g.k > 1 ? 4 : 0) + (premerge_used(g) ? 1 : 0) + 1;
 }
 
 namespace {

@@ -126,6 +126,9 @@ size_t carve(const moba::Geom& g, char* base, moba::Work* w) {
   x.rows = (int32_t*)take(sizeof(int32_t) * (size_t)moba::past_tiles(g) * moba::kPastTileRows);
   x.part_o = (__half*)take(sizeof(__half) * (size_t)g.R * g.D);
   x.part_lse = (float*)take(sizeof(float) * (size_t)g.R);
+  const size_t nmerged = moba::premerge_used(g) ? (size_t)g.T * g.Hq : 0;
+  x.merged_o = (__half*)take(sizeof(__half) * nmerged * g.D);
+  x.merged_lse = (float*)take(sizeof(float) * nmerged);
   x.kbar = (float*)take(sizeof(float) * (size_t)g.num_seqs * g.MB * g.Hkv * g.D);
   x.sel = (int32_t*)take(sizeof(int32_t) * (size_t)g.T * g.Hq * g.k);
   x.kbar_hi = (__nv_bfloat16*)take(2 * (size_t)g.num_seqs * g.MB * g.Hkv * g.D);

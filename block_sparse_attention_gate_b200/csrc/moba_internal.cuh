@@ -30,6 +30,13 @@ struct Geom {
   int* err;           // device error word (bounded waits that gave up), never null
 };
 
+// Rows with more than kPremergeMinPartials - 1 past partials (top_k - 1 >= 3) get them
+// folded by a separate pass before the own-block kernel.
+constexpr int kPremergeMinPartials = 3;
+__host__ __device__ inline bool premerge_used(const Geom& g) {
+  return g.T > 0 && g.k - 1 >= kPremergeMinPartials;
+}
+
 // Upper bound on the past-block attention tiles (kPastTileRows rows each): every bucket's
 // last tile may be partial.
 __host__ __device__ inline int64_t past_tiles(const Geom& g) {
@@ -62,6 +69,8 @@ struct Work {
   int32_t* rows;      // [past_tiles(g) * kPastTileRows] routed partial ids, tile by tile (-1: empty)
   __half* part_o;     // [R, D] normalised partial outputs (fp16)
   float* part_lse;    // [R] partial log-sum-exp
+  __half* merged_o;   // [T * Hq, D] folded partials (only when premerge_used)
+  float* merged_lse;  // [T * Hq]
   float* kbar;        // [num_seqs, MB, Hkv, D] (used by moba_fwd when the caller passes none)
   __nv_bfloat16* kbar_hi;  // [num_seqs, MB, Hkv, D] bf16 rn(Kbar) for the tensor-core gate
   __nv_bfloat16* kbar_lo;  // [num_seqs, MB, Hkv, D] bf16 rn(Kbar - hi)
