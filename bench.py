@@ -12,6 +12,9 @@ Besides the headline workload (1M tokens by default) the line carries
   * ``dense_causal``: dense causal attention on the same GPU (torch SDPA, outside the
     MoBA timed region) at the headline workload and at 32K MHA, and the library's own
     full mode (top_k >= number of blocks) at 32K MHA;
+  * ``backward``, ``decode``, ``mask_based``: the backward pass at the headline workload,
+    gated decode over its keys and values as KV caches (with dense decode beside it), and
+    the mask-based form against the efficient path at 32K;
   * ``e2e``: the public host-buffer call with its host<->device copies timed;
   * ``cpu_baseline``: the fp64 oracle on the host cores on a bounded row sample.
 
@@ -417,6 +420,161 @@ def dense_comparators(mp_main: MobaPass, main_ms: float, dev, dist) -> dict:
     return res
 
 
+def time_backward(mp: MobaPass, dist, steps: int = 2, warmup: int = 1) -> dict:
+    """The backward pass (moba_attn_bwd) at the workload of `mp`, after its forward: selection
+    held fixed, dO synthetic N(0,1).  FLOPs by the usual accounting, 2.5x the forward
+    attention's (five matrix products against two; the kernels recompute S and dP once more)."""
+    import torch
+    mb = mp.mb
+    stream = torch.cuda.current_stream(mp.dev)
+    mp.step(stream)
+    dO = torch.randn(mp.Q.shape, dtype=torch.bfloat16, device=mp.dev,
+                     generator=torch.Generator(device=mp.dev).manual_seed(7))
+    ws = torch.empty(max(mb.moba_bwd_workspace_size(mp.p), 256), dtype=torch.uint8, device=mp.dev)
+    dQ, dK, dV = torch.empty_like(mp.Q), torch.empty_like(mp.K), torch.empty_like(mp.V)
+
+    def run():
+        mb.moba_attn_bwd(mp.p, mp.Q, mp.K, mp.V, mp.O, mp.LSE, dO, mp.sel, ws, dQ, dK, dV, stream)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize(mp.dev)
+    if dist is not None:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        run()
+    b.record(stream)
+    torch.cuda.synchronize(mp.dev)
+    ms = max_over_ranks(a.elapsed_time(b) / steps, dist, mp.dev)
+    fl = flop_counts(mp.w, mp.routed_rows())
+    bw_flops = int(2.5 * fl["attn"])
+    del ws, dQ, dK, dV, dO
+    torch.cuda.empty_cache()
+    return {"ms": ms, "steps": steps, "warmup": warmup, "flops": bw_flops,
+            "tflops": bw_flops / (ms / 1e3) / 1e12, "workload": workload_desc(mp.w),
+            "flop_accounting": "2.5 x forward attention FLOPs (S, dP, dV, dK, dQ products)"}
+
+
+def time_decode(mp: MobaPass, dist, peaks: dict, nseq: int = 8, reps: int = 20) -> dict:
+    """Gated decode over the headline workload's keys and values seen as the KV caches of
+    `nseq` sequences of equal length (the newest token of each is the query), next to dense
+    decode (torch SDPA over every cached key) on the same caches."""
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    mb, w = mp.mb, mp.w
+    T = w.total_tokens
+    L = T // nseq
+    cu = np.arange(nseq + 1, dtype=np.int32) * L
+    p = mb.MobaParams(cu, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.top_k)
+    K, V = mp.K[:nseq * L], mp.V[:nseq * L]
+    Qd = mp.Q[torch.as_tensor(cu[1:] - 1, device=mp.dev, dtype=torch.long)].contiguous()
+    kbar = torch.empty(p.kbar_elems, dtype=torch.float32, device=mp.dev)
+    mb.moba_pool_keys(p, K, kbar)
+    ws = torch.empty(max(mb.moba_decode_workspace_size(p), 256), dtype=torch.uint8, device=mp.dev)
+    sel = torch.empty((nseq, w.num_q_heads, w.top_k), dtype=torch.int32, device=mp.dev)
+    O = torch.empty_like(Qd)
+    LSE = torch.empty((nseq, w.num_q_heads), dtype=torch.float32, device=mp.dev)
+    stream = torch.cuda.current_stream(mp.dev)
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(mp.dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(mp.dev)
+        return a.elapsed_time(b) / n
+
+    ms = timed(lambda: mb.moba_decode_fwd(p, Qd, K, V, kbar, ws, O, LSE, sel=sel, stream=stream), reps)
+    ms = max_over_ranks(ms, dist, mp.dev)
+    # algorithmic bytes: the distinct selected blocks' keys and values per (sequence, KV head)
+    # (the own block up to the new token), the pooled keys the gate reads, Q and O
+    s_np = sel.cpu().numpy()
+    G, bs, D = w.num_q_heads // w.num_kv_heads, w.block_size, w.head_dim
+    own = (L - 1) // bs
+    nbytes = 0
+    for sq in range(nseq):
+        for g in range(w.num_kv_heads):
+            blocks = set(int(b) for b in s_np[sq, g * G:(g + 1) * G].ravel() if b >= 0)
+            for b in blocks:
+                nbytes += (L - b * bs if b == own else bs) * D * 2 * 2
+    nbytes += nseq * w.num_kv_heads * own * D * 4 + 2 * Qd.numel() * 2
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    res = {"workload": "%d sequences x %d cached tokens, Hq=%d Hkv=%d D=%d block_size=%d top_k=%d (the headline "
+                       "workload's keys and values)" % (nseq, L, w.num_q_heads, w.num_kv_heads, D, bs, w.top_k),
+           "ms": ms, "tokens_per_s": nseq / (ms / 1e3), "algorithmic_bytes": nbytes,
+           "achieved_gbs": nbytes / (ms / 1e3) / 1e9, "hbm_peak_gbs": hbm,
+           "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / hbm, "launches": 3}
+    # dense decode: every cached key, torch SDPA (one query per sequence and head)
+    q4 = Qd.unsqueeze(2)  # [B, Hq, 1, D]
+    k4 = K.view(nseq, L, w.num_kv_heads, D).permute(0, 2, 1, 3)
+    v4 = V.view(nseq, L, w.num_kv_heads, D).permute(0, 2, 1, 3)
+    k4 = k4.repeat_interleave(G, dim=1).contiguous()
+    v4 = v4.repeat_interleave(G, dim=1).contiguous()
+    dense = None
+    for backend, name in ((SDPBackend.CUDNN_ATTENTION, "cudnn"), (SDPBackend.FLASH_ATTENTION, "flash"),
+                          (SDPBackend.EFFICIENT_ATTENTION, "efficient")):
+        try:
+            with sdpa_kernel([backend]):
+                dms = timed(lambda: F.scaled_dot_product_attention(q4, k4, v4), reps)
+            dense = (max_over_ranks(dms, dist, mp.dev), name)
+            break
+        except RuntimeError:
+            continue
+    if dense is not None:
+        dbytes = 2 * nseq * w.num_kv_heads * L * D * 2
+        res["dense_decode"] = {"impl": "torch SDPA (%s) over every cached key" % dense[1], "ms": dense[0],
+                               "kv_bytes_per_kv_head": dbytes, "moba_speedup": dense[0] / ms}
+    del k4, v4, ws, kbar
+    torch.cuda.empty_cache()
+    return res
+
+
+def time_mask_based(dev, dist) -> dict:
+    """The mask-based form (moba_attn_naive: every causal key scored, unselected blocks
+    masked) against the efficient path (route + past blocks + own block), on the same
+    selection: at 32K tokens with one head, block 2048, top_k 3 (the configuration of the
+    pages' efficient-versus-naive comparison) and at 32K MHA (32 heads)."""
+    import torch
+    out = {}
+    for name, w in (("32k_1head", synth.Workload("mask32k_h1", [32768], 1, 1, 128, 2048, 3, seed=1006,
+                                                 rope_theta=500000.0)),
+                    ("mha32k", synth.CONFIGS["mha32k"])):
+        mp = MobaPass(w, dev)
+        stream = torch.cuda.current_stream(dev)
+        mb, p = mp.mb, mp.p
+        mp.step(stream)
+        On, Ln = torch.empty_like(mp.O), torch.empty_like(mp.LSE)
+
+        def timed(fn, n=10):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            return a.elapsed_time(b) / n
+
+        eff = timed(lambda: mb.moba_attn_fwd(p, mp.Q, mp.K, mp.V, mp.sel, mp.ws, mp.O, mp.LSE, stream))
+        nv = timed(lambda: mb.moba_attn_naive(p, mp.Q, mp.K, mp.V, mp.sel, On, Ln, stream))
+        eff, nv = max_over_ranks(eff, dist, dev), max_over_ranks(nv, dist, dev)
+        out[name] = {"workload": workload_desc(w), "efficient_ms": eff, "mask_based_ms": nv,
+                     "speedup": nv / eff, "dense_causal_flops": dense_causal_flops(w),
+                     "mask_based_tflops": dense_causal_flops(w) / (nv / 1e3) / 1e12}
+        del mp, On, Ln
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | None:
     import torch
     import block_sparse_attention_gate_b200 as mb
@@ -514,6 +672,10 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
                           if name != w.name}
     if not args.no_dense:
         res["dense_causal"] = dense_comparators(mp, ms_step, dev, dist)
+    if not args.no_extra:
+        res["backward"] = time_backward(mp, dist)
+        res["decode"] = time_decode(mp, dist, peaks)
+        res["mask_based"] = time_mask_based(dev, dist)
     if rank == 0 and world == 1 and not args.no_cpu:
         Kh = host["k"].view(torch.int16).numpy().view(np.uint16)
         Vh = host["v"].view(torch.int16).numpy().view(np.uint16)
@@ -573,12 +735,20 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-side", action="store_true", help="skip the other long-context workloads")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense causal comparators")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the backward, decode and mask-based records")
+    ap.add_argument("--scale", type=float, default=1.0,
+                    help="scale the workload's sequence lengths (for small profiling captures)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=4.0)
     args = ap.parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     w = synth.CONFIGS[args.config]
+    if args.scale != 1.0:
+        import dataclasses
+        lens = [max(1, int(round(L * args.scale))) for L in w.seqlens]
+        w = dataclasses.replace(w, name="%s_x%g" % (w.name, args.scale), seqlens=lens)
     if args.impl == "reference":
         res = run_reference(args, w, rank, world)
         if res is not None:
