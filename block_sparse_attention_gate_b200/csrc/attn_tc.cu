@@ -1049,6 +1049,7 @@ cudaError_t launch_past_persistent(const Geom& g, const __nv_bfloat16* K, const 
   attn_past_persistent_kernel<D><<<grid, kThreads, smem, st>>>(tk, tv, a);
   return cudaGetLastError();
 }
+
 }  // namespace
 
 cudaError_t launch_attn_past(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
@@ -1083,7 +1084,7 @@ __global__ void __launch_bounds__(256) premerge_kernel(Geom g, const int32_t* __
                                                        const __half* __restrict__ part_o,
                                                        const float* __restrict__ part_lse, __half* __restrict__ mo,
                                                        float* __restrict__ mlse) {
-  constexpr int kDL = D / 32;
+  constexpr int kDL = D / 32;  // elements of a partial row per lane
   const int lane = threadIdx.x & 31;
   const int64_t rows = (int64_t)g.T * g.Hq;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -1092,31 +1093,48 @@ __global__ void __launch_bounds__(256) premerge_kernel(Geom g, const int32_t* __
     const int32_t t = (int32_t)(row / g.Hq);
     const int s = find_seq(g, t);
     const int i = (t - seq_start(g, s)) / g.bs;
-    // the row's past partials: the chosen past blocks fill the first np slots
-    int np = 0;
-    bool run = true;
-    for (int q = 0; q < km1; ++q) {
-      const int32_t b = __ldg(sel + row * g.k + 1 + q);
-      run = run && b >= 0 && b < i;
-      np += run ? 1 : 0;
-    }
-    if (np < 2) continue;
     const int64_t base = row * km1;
-    float M = -INFINITY;
-    for (int q = 0; q < np; ++q) M = fmaxf(M, __ldg(part_lse + base + q));
-    float L = 0.f, acc[kDL];
+    // One round trip per row: lane q reads slot q's block and LSE, and every lane reads its
+    // share of all km1 partial rows at once (in bounds whether or not a slot is used; the
+    // unused ones are excluded by a select below, never multiplied in).
+    const int32_t b = lane < km1 ? __ldg(sel + row * g.k + 1 + lane) : -1;
+    const float lq = lane < km1 ? __ldg(part_lse + base + lane) : -INFINITY;
+    uint32_t raw[kMaxTopK - 1][kDL / 2];
+#pragma unroll
+    for (int q = 0; q < kMaxTopK - 1; ++q) {
+      const __half* src = part_o + (base + (q < km1 ? q : 0)) * D + lane * kDL;
+      if constexpr (kDL == 4) {
+        const uint2 v = q < km1 ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0u, 0u);
+        raw[q][0] = v.x;
+        raw[q][1] = v.y;
+      } else {
+        raw[q][0] = q < km1 ? __ldg(reinterpret_cast<const uint32_t*>(src)) : 0u;
+      }
+    }
+    // the chosen past blocks fill the first np slots
+    const uint32_t bad = __ballot_sync(0xffffffffu, !(b >= 0 && b < i));
+    const int np = min(km1, __ffs(bad) - 1);
+    if (np < 2) continue;  // the own-block kernel reads a lone partial where it is
+    float M = lane < np ? lq : -INFINITY;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float wl = lane < np ? __expf(lq - M) : 0.f;
+    float L = wl;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    float acc[kDL];
 #pragma unroll
     for (int x = 0; x < kDL; ++x) acc[x] = 0.f;
-#pragma unroll 4
-    for (int q = 0; q < np; ++q) {
-      const float w = __expf(__ldg(part_lse + base + q) - M);
-      L += w;
-      const __half2* src = reinterpret_cast<const __half2*>(part_o + (base + q) * D + lane * kDL);
 #pragma unroll
-      for (int x = 0; x < kDL / 2; ++x) {
-        const float2 f = __half22float2(src[x]);
-        acc[2 * x] = fmaf(w, f.x, acc[2 * x]);
-        acc[2 * x + 1] = fmaf(w, f.y, acc[2 * x + 1]);
+    for (int q = 0; q < kMaxTopK - 1; ++q) {
+      const float w = __shfl_sync(0xffffffffu, wl, q);
+      if (q < np) {
+#pragma unroll
+        for (int x = 0; x < kDL / 2; ++x) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&raw[q][x]));
+          acc[2 * x] = fmaf(w, f.x, acc[2 * x]);
+          acc[2 * x + 1] = fmaf(w, f.y, acc[2 * x + 1]);
+        }
       }
     }
     const float inv = 1.f / L;
@@ -1132,8 +1150,7 @@ cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_b
                              const __nv_bfloat16* V, const int32_t* sel, const Work& w,
                              __nv_bfloat16* O, float* LSE, cudaStream_t st) {
   if (g.T == 0) return cudaSuccess;
-  int head_pairs = 0;
-  const dim3 grid = own_grid(g, &head_pairs);
+  const int head_pairs = (g.G % 2 == 0) ? 1 : 0;
   int premerged = 0;
   if (premerge_used(g)) {
     const int64_t rows = (int64_t)g.T * g.Hq;
@@ -1145,6 +1162,8 @@ cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_b
     if (e != cudaSuccess) return e;
     premerged = 1;
   }
+  int hp = 0;
+  const dim3 grid = own_grid(g, &hp);
   if (g.D == 64) return launch_tc<64, kModeOwn>(g, Q, K, V, sel, w, O, LSE, grid, head_pairs, st, premerged);
   return launch_tc<128, kModeOwn>(g, Q, K, V, sel, w, O, LSE, grid, head_pairs, st, premerged);
 }

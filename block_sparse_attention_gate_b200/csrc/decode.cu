@@ -206,22 +206,32 @@ __global__ void __launch_bounds__(kAttnWarps * 32)
     m = m_new;
 #pragma unroll
     for (int x = 0; x < kDL; ++x) o[x] *= alpha;
-    for (int j = 0; j < nk; ++j) {
-      const float pj = __shfl_sync(0xffffffffu, pz, j);
-      const __nv_bfloat16* vp = vbase + (int64_t)(r0 + j) * kv_stride;
-      if constexpr (kDL == 4) {
-        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(vp));
-        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-        const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
-        o[0] = fmaf(pj, a.x, o[0]);
-        o[1] = fmaf(pj, a.y, o[1]);
-        o[2] = fmaf(pj, c.x, o[2]);
-        o[3] = fmaf(pj, c.y, o[3]);
-      } else {
-        const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(vp));
-        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw));
-        o[0] = fmaf(pj, a.x, o[0]);
-        o[1] = fmaf(pj, a.y, o[1]);
+    // the value rows of the round, eight at a time: the eight loads are in flight together
+    // (a loop, not unrolled, so the registers stay few and several CTAs fit on an SM)
+#pragma unroll 1
+    for (int j0 = 0; j0 < 32; j0 += 8) {
+      uint32_t vr[8][kDL / 2];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const __nv_bfloat16* vp = vbase + (int64_t)(r0 + j0 + j) * kv_stride;
+        if constexpr (kDL == 4) {
+          uint2 raw = make_uint2(0u, 0u);
+          if (j0 + j < nk) raw = __ldg(reinterpret_cast<const uint2*>(vp));
+          vr[j][0] = raw.x;
+          vr[j][1] = raw.y;
+        } else {
+          vr[j][0] = j0 + j < nk ? __ldg(reinterpret_cast<const uint32_t*>(vp)) : 0u;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float pj = __shfl_sync(0xffffffffu, pz, j0 + j);  // 0 for keys past the block's end
+#pragma unroll
+        for (int x = 0; x < kDL / 2; ++x) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vr[j][x]));
+          o[2 * x] = fmaf(pj, f.x, o[2 * x]);
+          o[2 * x + 1] = fmaf(pj, f.y, o[2 * x + 1]);
+        }
       }
     }
   }
