@@ -1,9 +1,7 @@
-// MoBA block attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+// MoBA own-block attention + merge, and the mask-based form, on the 5th-generation tensor
+// cores (tcgen05 + TMEM + TMA).  (The past blocks are in attn_past.cu.)
 //
-// Three modes share one kernel body:
-//   past : a CTA takes two tiles of 128 routed query rows of one bucket (KV head g,
-//          sequence s, past block b), attends the whole block (bs keys; a past block is
-//          complete and fully visible) and writes normalised partials (fp16) + LSE (fp32).
+// Two modes share the body of attn_tc_kernel:
 //   own  : a CTA takes two tiles of 128 tokens (two heads, or two consecutive tiles of one
 //          head) inside one block.  Each row's past partials are merged FIRST: they become
 //          the starting state (m, l, O) of the online softmax, which then runs over the
@@ -30,71 +28,11 @@
 #include <cudaTypedefs.h>
 #include <float.h>
 
-#include "moba_internal.cuh"
-#include "sm100.cuh"
+#include "attn_common.cuh"
 
 namespace moba {
 
 namespace {
-
-constexpr int kThreads = 384;  // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA, 10-11 idle
-// Register split (setmaxnreg): the kernel is compiled for kLaunchRegs per thread; the third
-// warpgroup gives registers back so the two softmax warpgroups can hold a full S row.
-// 2 * 128 * kSoftmaxRegs + 128 * kOtherRegs must not exceed 384 * kLaunchRegs (checked on
-// the host against the compiled register count before every launch).
-constexpr uint32_t kLaunchRegs = 168;
-constexpr uint32_t kSoftmaxRegs = 216;
-constexpr uint32_t kOtherRegs = 72;
-static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= 384 * kLaunchRegs, "register split too large");
-constexpr int kRows = 128;     // query rows per tile (M); two tiles per CTA
-constexpr int kBN = 128;       // keys per chunk (N of S, K of PV)
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;      // S of tile t at kColS + 128 t
-constexpr uint32_t kColP = 0;      // P of tile t (bf16 pairs) aliased at S + 0 .. S + 63
-constexpr uint32_t kColO = 256;    // O of tile t at kColO + 128 t
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleLog2 = 8.f;  // rescale O only when a row max grows by more than 2^8
-
-// 2^x for a pair on the FMA pipe, for a share of the exponentials that would otherwise all
-// queue on the MUFU unit: x = j + f with j = rint(x) (the 1.5 * 2^23 rounding trick) and
-// f in [-0.5, 0.5]; 2^f from a degree-3 polynomial (relative error 7.5e-5; coefficients from
-// our own iteratively reweighted least-squares fit of 2^f on that interval), 2^j added into
-// the exponent field.  x is clamped to >= -126 so the exponent never wraps; below 2^-24 the
-// result only has to be negligible next to the row sum, as it is.
-constexpr int kPolyNum = 1, kPolyDen = 4;  // pairs (pair index mod kPolyDen) < kPolyNum use it
-__device__ __forceinline__ void exp2_poly2(float& p0, float& p1, float x0, float x1) {
-  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  float t0, t1, r0, r1, f0, f1, q0, q1;
-  add2(t0, t1, x0, x1, kRound, kRound);
-  add2(r0, r1, t0, t1, -kRound, -kRound);
-  fma2(f0, f1, r0, r1, -1.f, -1.f, x0, x1);
-  fma2(q0, q1, f0, f1, 0.05517132207751274f, 0.05517132207751274f, 0.24261054396629333f, 0.24261054396629333f);
-  fma2(q0, q1, q0, q1, f0, f1, 0.6932609677314758f, 0.6932609677314758f);
-  fma2(q0, q1, q0, q1, f0, f1, 0.9999281167984009f, 0.9999281167984009f);
-  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
-
-struct AttnArgs {
-  Geom g;
-  const __nv_bfloat16* Q;
-  const int32_t* sel;
-  const int32_t* tile_off;
-  const int32_t* tile_bucket;
-  const int32_t* rows;
-  __half* part_o;
-  float* part_lse;
-  __nv_bfloat16* O;
-  float* LSE;
-  int own_head_pairs;  // own mode: tiles are heads (2p, 2p+1) of one group (else query tiles 2p, 2p+1)
-  int premerged;       // own mode: rows with two or more past partials have them folded in mo/mlse
-  const __half* mo;    // [T * Hq, D] folded partial of each such row
-  const float* mlse;   // [T * Hq] its LSE
-};
-
 template <int D>
 struct Layout {
   static constexpr int kTile = kRows * D * 2;  // bytes of a [128 x D] bf16 tile
@@ -113,15 +51,13 @@ enum Bar {
 
 // One tile's row source and causal geometry.
 struct TileInfo {
-  int64_t qrow_base;  // own mode: Q row of token q0 (t * Hq + h) ...
-  int32_t q0;         // own mode: first token
-  int h;              // own mode: query head
-  int nrows;          // valid rows (0..128)
-  int diag;           // own mode: index of the diagonal chunk
-  int32_t row_start;  // past mode: first routed position
+  int32_t q0;  // first token
+  int h;       // query head
+  int nrows;   // valid rows (0..128)
+  int diag;    // index of the diagonal chunk
 };
 
-enum Mode : int { kModePast = 0, kModeOwn = 1, kModeNaive = 2 };
+enum Mode : int { kModeOwn = 1, kModeNaive = 2 };
 
 template <int D, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -134,34 +70,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kNumBars * 8);
   const Geom& g = a.g;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  constexpr bool kPast = kMode == kModePast;
   constexpr bool kNaive = kMode == kModeNaive;
-  constexpr bool kOwn = !kPast;  // tiles of consecutive tokens that end with the final O and LSE
 
   // ------------------------------------------------------------- work item
   int gk, s, i_blk = 0, nchunks;
   int32_t key0;
   TileInfo ti[2];
-  if constexpr (!kOwn) {
-    // The routed rows are laid out tile by tile (kPastTileRows slots per tile, -1 in the
-    // slots past a bucket's last row), so a tile needs only its bucket and its own slots.
-    const int32_t tile = (int32_t)blockIdx.x;
-    const int32_t total = __ldg(a.tile_off + g.nbk);
-    const int64_t lo = __ldg(a.tile_bucket + tile);  // in bounds for every launched tile
-    if (tile >= total) return;
-    const int32_t b = (int32_t)(lo % g.MB);
-    s = (int)((lo / g.MB) % g.num_seqs);
-    gk = (int)(lo / ((int64_t)g.MB * g.num_seqs));
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      ti[t].row_start = tile * kPastTileRows + t * kRows;
-      ti[t].nrows = kRows;  // empty slots hold -1
-      ti[t].diag = 1 << 30;
-      ti[t].qrow_base = 0; ti[t].q0 = 0; ti[t].h = 0;
-    }
-    key0 = seq_start(g, s) + b * g.bs;
-    nchunks = g.bs / kBN;
-  } else {
+  {
     const int per_blk = g.bs / kRows;
     s = blockIdx.y;
     const int32_t ts = seq_start(g, s), te = seq_end(g, s);
@@ -186,7 +101,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ti[t].q0 = q0;
         ti[t].nrows = min(kRows, te - q0);
         ti[t].diag = qt;
-        ti[t].row_start = 0;
       }
       nchunks = qt + 1;
     } else {
@@ -209,7 +123,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ti[t].q0 = q0 + t * kRows;
         ti[t].nrows = (t == 0 || has1) ? max(0, min(kRows, te - ti[t].q0)) : 0;
         ti[t].diag = 2 * qp + t;
-        ti[t].row_start = 0;
       }
       nchunks = has1 ? qt1 + 1 : 2 * qp + 1;
     }
@@ -232,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int np = 0;                 // own mode: past partials of this thread's row
   float pmax = -INFINITY;     // own mode: their largest LSE, log2 units
   bool folded = false;        // own mode: the row's partials come folded (one partial in mo/mlse)
-  if (kOwn && !kNaive && warp < 8) {
+  if (!kNaive && warp < 8) {
     const int t = warp >> 2, r = tid & (kRows - 1);
     if (r < ti[t].nrows) {
       const int64_t qrow = (int64_t)(ti[t].q0 + r) * g.Hq + ti[t].h;
@@ -250,21 +163,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         for (int q = 0; q < np; ++q) pmax = fmaxf(pmax, __ldg(a.part_lse + qrow * (g.k - 1) + q) * kLog2e);
       }
-    }
-  }
-  // Past mode: the softmax threads look up their routed rows and start the Q gather before
-  // the setup below.
-  int32_t e = -1;  // past mode: this thread's partial id (-1: empty slot)
-  if (kPast && warp < 8) {
-    const int t = warp >> 2, r = tid & (kRows - 1);
-    {
-      e = __ldg(a.rows + ti[t].row_start + r);
-      const int64_t qrow = e >= 0 ? e / (g.k - 1) : -1;
-      const __nv_bfloat16* src = qrow >= 0 ? a.Q + qrow * D : a.Q;
-      const uint32_t nb = qrow >= 0 ? 16u : 0u;  // zeros for empty slots
-      const uint32_t sQ = smem_u32(smem + L::kQ + t * L::kTile);
-#pragma unroll
-      for (int c = 0; c < D / 8; ++c) cp_async_16(sQ + sw128_offset(r, c, kRows), src + c * 8, nb);
     }
   }
   auto load_k = [&](int j) {  // K of chunk j into stage j & 1 (TMA producer)
@@ -291,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
   }
   if (tid == 0) {
-    mbar_init(&bars[kQFull], kOwn ? 1 : 2 * kRows);  // own, naive: one TMA transaction; past: every row's gather
+    mbar_init(&bars[kQFull], 1);  // one TMA transaction
     for (int q = 0; q < 2; ++q) {
       mbar_init(&bars[kKFull0 + q], 1);
       mbar_init(&bars[kKEmpty0 + q], 1);
@@ -315,20 +213,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = warp >> 2;           // tile
     const int r = tid & (kRows - 1);   // row = TMEM lane
     const TileInfo& T_ = ti[t];
-    int64_t qrow = -1;  // own mode: this row's (token, head) row of Q, O and LSE
-    if (kOwn && r < T_.nrows) qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
-    if constexpr (!kOwn) {  // this row's Q gather (issued before the setup) has landed
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(&bars[kQFull]);
-    }
+    int64_t qrow = -1;  // this row's (token, head) row of Q, O and LSE
+    if (r < T_.nrows) qrow = (int64_t)(T_.q0 + r) * g.Hq + T_.h;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + kColS + t * kBN;
     const uint32_t tP = tS + kColP;
     const uint32_t tO = tmem + lane_off + kColO + t * 128;
     const float c2 = g.scale_log2;
     float m = -INFINITY, l = 0.f;
-    if constexpr (kOwn) {
+    {
       // Merge first: the row's past partials (normalised O_q and LSE_q, written by the
       // past-block attention before this kernel runs) become the starting state of the
       // online softmax, in its log2 units: m = max_q LSE_q log2(e), w_q = 2^(LSE_q log2(e) - m),
@@ -393,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
       // scaled-logit row max (log2 units); the causal mask applies to the diagonal chunk only
       // (keys after the diagonal chunk, in the query-tile-pair layout, are all masked)
-      bool masked = kOwn && j >= T_.diag;
-      int lim = (kOwn && j == T_.diag) ? r + 1 : (masked ? 0 : kBN);
+      bool masked = j >= T_.diag;
+      int lim = j == T_.diag ? r + 1 : (masked ? 0 : kBN);
       if constexpr (kNaive) {  // keys of a block the row did not select get zero weight
         const int32_t blk = (j * kBN) / g.bs;
         bool on = false;
@@ -425,9 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // running max: rescale the TMEM accumulator only when it grows by more than 2^8
       // (p <= 256 otherwise, harmless in fp32 sums and bf16 P).  At this point the previous
       // PV of this tile has completed: the MMA that produced this S was issued after it.
-      if (kPast && j == 0) {
-        m = mx;
-      } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {  // own mode: m may start at -inf
+      if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {  // m may start at -inf
         const float m_new = fmaxf(m, mx);
         // naive mode: a row whose keys so far were all masked has m = m_new = -inf (its O and
         // l are still zero); its factor must not become 2^(-inf + inf)
@@ -503,10 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const float lse_row = (m + __log2f(l)) * kLn2;
-      // Past mode: the normalised partial row (fp16: its rounding, at most 2^-11 of |O| per
-      // element, is far below the bf16 rounding of the final output) and its LSE, at the
-      // row's partial id.  Own mode: the final O row (bf16) and LSE: the past partials were
-      // merged in at the start.
+      // The final O row (bf16) and LSE: the past partials were merged in at the start.
       // Each thread stages its own row (rows padded by 16 bytes so the row-per-thread 16-byte
       // writes spread over the banks) and hands it to the TMA engine as one bulk copy.  The
       // copies drain to memory on their own; the thread only waits until the engine has read
@@ -525,33 +413,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
           const float v0 = __uint_as_float(o[x]) * inv_l, v1 = __uint_as_float(o[x + 1]) * inv_l;
-          if constexpr (kOwn) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
-            hv[x >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
-          } else {
-            const __half2 h2v = __floats2half2_rn(v0, v1);
-            hv[x >> 1] = *reinterpret_cast<const uint32_t*>(&h2v);
-          }
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
+          hv[x >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
         }
 #pragma unroll
         for (int x = 0; x < 16; x += 4)
           *reinterpret_cast<uint4*>(srow + c * 64 + x * 4) = make_uint4(hv[x], hv[x + 1], hv[x + 2], hv[x + 3]);
       }
-      void* dst = nullptr;
-      if constexpr (kOwn) {
-        if (qrow >= 0) {
-          a.LSE[qrow] = lse_row;
-          dst = a.O + qrow * D;
-        }
-      } else {
-        if (e >= 0) {
-          a.part_lse[e] = lse_row;
-          dst = a.part_o + (int64_t)e * D;
-        }
-      }
-      if (dst) {
+      if (qrow >= 0) {
+        a.LSE[qrow] = lse_row;
         fence_proxy_async_smem();
-        bulk_store_s2g(dst, smem_u32(srow), D * 2);
+        bulk_store_s2g(a.O + qrow * D, smem_u32(srow), D * 2);
         bulk_commit();
         bulk_wait_read_all();
       }
@@ -561,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      if constexpr (kOwn) {  // both Q tiles: 128 consecutive tokens of one head each
+      {  // both Q tiles: 128 consecutive tokens of one head each
         prefetch_tmap(&tmQ);
         mbar_expect_tx(&bars[kQFull], 2 * L::kTile);
 #pragma unroll
@@ -603,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk)
         mma_bf16_ts_warp(tmem + kColO + t * 128, tmem + kColS + t * kBN + kColP + kk * 8,
-                         sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), idO, (kOwn || j > 0 || kk > 0) ? 1u : 0u);
+                         sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), idO, 1u);  // O starts from the merge
     };
     ok = mbar_wait_warp(&bars[kQFull], 0, g.err) && mbar_wait_warp(&bars[kKFull0], 0, g.err);
     if (ok) {
@@ -656,12 +528,8 @@ cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16
   CUtensorMap tq, tk, tv;
   cudaError_t e = make_rows_map(&tk, K, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
-  if (kMode != kModePast) {
-    e = make_rows_map(&tq, Q, (uint64_t)g.T, g.Hq, D, kRows);
-    if (e != cudaSuccess) return e;
-  } else {
-    tq = tk;  // unused: past mode gathers its Q rows
-  }
+  e = make_rows_map(&tq, Q, (uint64_t)g.T, g.Hq, D, kRows);
+  if (e != cudaSuccess) return e;
   e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
   AttnArgs a{g, Q, sel, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, O, LSE, head_pairs, premerged,
@@ -679,385 +547,7 @@ cudaError_t launch_tc(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16
 }
 
 
-// Warp-wide MMA issue with 32-bit descriptor words: every shared-memory descriptor here has
-// SBO 1024, version 1 and the 128-byte swizzle, so its upper word is the constant 0x40004040.
-__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes) {
-  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
-}
-__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b32 hi;\n\t.reg .b64 da, db;\n\t"
-      "mov.b32 hi, 0x40004040;\n\tmov.b64 da, {%1, hi};\n\tmov.b64 db, {%2, hi};\n\t"
-      "elect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b32 hi;\n\t.reg .b64 db;\n\t"
-      "mov.b32 hi, 0x40004040;\n\tmov.b64 db, {%2, hi};\n\t"
-      "elect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(acc)
-      : "memory");
-}
-// ===================================================================== persistent past mode
-// One CTA per SM walks the tile pairs blockIdx.x, blockIdx.x + gridDim.x, ...  Barrier phases
-// run on across items: K/V stages and the S/P barriers count chunks globally (J), the Q, O
-// and O-drained barriers count items (n).  The next item's routed rows are read early and its
-// Q gather goes out as soon as this item's last S of the tile has completed; its first S MMAs
-// then overlap this item's epilogue.  The epilogue stages 8 rows per warp at a time in a
-// dedicated region (the Q and K/V buffers already hold the next item's data).
-enum PBar {
-  pQFull = 0, pKFull0, pKFull1, pKEmpty0, pKEmpty1, pVFull0, pVFull1, pVEmpty0, pVEmpty1,
-  pSFull0, pSFull1, pPFull0, pPFull1, pOFull0, pOFull1, pODrained0, pODrained1, pDone, pNumBars
-};
-template <int D>
-struct PLayout {
-  static constexpr int kTile = kRows * D * 2;
-  static constexpr int kQ = 0;
-  static constexpr int kK0 = kQ + 2 * kTile;
-  static constexpr int kV0 = kK0 + 2 * kTile;
-  static constexpr int kBar = kV0 + 2 * kTile;
-  static constexpr int kStgRow = D * 2 + 16;  // fp16 row, padded by 16 bytes
-  static constexpr int kStg = kBar + 256;     // 8 warps x 8 rows
-  static constexpr int kBytes = kStg + 8 * 8 * kStgRow;
-  static constexpr int kAlloc = kBytes + 1024;
-};
-
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-    attn_past_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                                AttnArgs a) {
-  using L = PLayout<D>;
-  static_assert(pNumBars * 8 + 4 <= 256, "barrier area");
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + pNumBars * 8);
-  const Geom& g = a.g;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int32_t total = __ldg(a.tile_off + g.nbk);
-  const int32_t first = (int32_t)blockIdx.x, stride = (int32_t)gridDim.x;
-  if (first >= total) return;
-  const int nitems = (total - 1 - first) / stride + 1;
-  const int nchunks = g.bs / kBN;
-
-  // ------------------------------------------------------------- item 0's rows and Q gather
-  int32_t e_cur = -1;
-  auto gather_q = [&](int t, int r, int32_t e) {
-    const int64_t qrow = e >= 0 ? e / (g.k - 1) : -1;
-    const __nv_bfloat16* src = qrow >= 0 ? a.Q + qrow * D : a.Q;
-    const uint32_t nb = qrow >= 0 ? 16u : 0u;
-    const uint32_t sQ = smem_u32(smem + L::kQ + t * L::kTile);
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) cp_async_16(sQ + sw128_offset(r, c, kRows), src + c * 8, nb);
-  };
-  if (warp < 8) {
-    const int t = warp >> 2, r = tid & (kRows - 1);
-    e_cur = __ldg(a.rows + (int64_t)first * kPastTileRows + t * kRows + r);
-    gather_q(t, r, e_cur);
-  }
-
-  // ------------------------------------------------------------- setup
-  if (warp == 9) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
-    tc_fence_before();
-  }
-  if (tid == 0) {
-    mbar_init(&bars[pQFull], 2 * kRows);
-    for (int q = 0; q < 2; ++q) {
-      mbar_init(&bars[pKFull0 + q], 1);
-      mbar_init(&bars[pKEmpty0 + q], 1);
-      mbar_init(&bars[pVFull0 + q], 1);
-      mbar_init(&bars[pVEmpty0 + q], 1);
-      mbar_init(&bars[pSFull0 + q], 1);
-      mbar_init(&bars[pPFull0 + q], kRows);
-      mbar_init(&bars[pOFull0 + q], 1);
-      mbar_init(&bars[pODrained0 + q], kRows);
-    }
-    mbar_init(&bars[pDone], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  bool ok = true;
-  if (warp >= 8) regs_dec<kOtherRegs>(); else regs_inc<kSoftmaxRegs>();
-
-  if (warp < 8) {
-    // ========================================================= softmax warpgroups
-    const int t = warp >> 2;
-    const int r = tid & (kRows - 1);
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_off + kColS + t * kBN;
-    const uint32_t tP = tS + kColP;
-    const uint32_t tO = tmem + lane_off + kColO + t * 128;
-    const float c2 = g.scale_log2;
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    mbar_arrive(&bars[pQFull]);
-    uint32_t J = 0;
-    for (int n = 0; n < nitems && ok; ++n) {
-      const bool has_next = n + 1 < nitems;
-      const int32_t e_next =
-          has_next ? __ldg(a.rows + (int64_t)(first + (n + 1) * stride) * kPastTileRows + t * kRows + r) : -1;
-      float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < nchunks && ok; ++j, ++J) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars[pSFull0 + t], J & 1, g.err));
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
-        tmem_wait_ld();
-        if (j == nchunks - 1 && has_next) gather_q(t, r, e_next);  // Q_t is free: its last S completed
-        float mv[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mv[q] = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int x = 0; x < 32; x += 2)
-            mv[(x >> 1) & 7] = max3(mv[(x >> 1) & 7], __uint_as_float(sr[c][x]), __uint_as_float(sr[c][x + 1]));
-        float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])), fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
-        mx *= c2;
-        if (j == 0) {
-          m = mx;
-        } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
-          const float m_new = fmaxf(m, mx);
-          const float alpha = ex2(m - m_new);
-          l *= alpha;
-          m = m_new;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(tO + c * 32, o);
-          }
-        }
-        float rv[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) rv[q] = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int c = 2 * cc + h2;
-#pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const int pi = x >> 1;
-              float u0, u1, p0, p1;
-              fma2(u0, u1, __uint_as_float(sr[c][x]), __uint_as_float(sr[c][x + 1]), c2, c2, -m, -m);
-              if (pi % kPolyDen < kPolyNum) {
-                exp2_poly2(p0, p1, u0, u1);
-              } else {
-                p0 = ex2(u0);
-                p1 = ex2(u1);
-              }
-              const int q = 2 * (pi & 3);
-              add2(rv[q], rv[q + 1], rv[q], rv[q + 1], p0, p1);
-              pk[16 * h2 + pi] = pack_bf16x2(p0, p1);
-            }
-          }
-          tmem_st32(tP + cc * 32, pk);
-        }
-        l += ((rv[0] + rv[1]) + (rv[2] + rv[3])) + ((rv[4] + rv[5]) + (rv[6] + rv[7]));
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars[pPFull0 + t]);
-      }
-      if (!ok) break;
-      if (has_next) {  // the next item's Q rows of this tile have landed
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(&bars[pQFull]);
-      }
-      // ------------------------------------------------------- epilogue of item n
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[pOFull0 + t], n & 1, g.err));
-      if (!ok) break;
-      tc_fence_after();
-      const float inv_l = 1.f / l;
-      const float lse_row = (m + __log2f(l)) * kLn2;
-      uint32_t hv[D / 2];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const __half2 h2v = __floats2half2_rn(__uint_as_float(o[x]) * inv_l, __uint_as_float(o[x + 1]) * inv_l);
-          hv[c * 16 + (x >> 1)] = *reinterpret_cast<const uint32_t*>(&h2v);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bars[pODrained0 + t]);  // O_t may now be overwritten by the next item
-      if (e_cur >= 0) a.part_lse[e_cur] = lse_row;
-      uint8_t* slot = smem + L::kStg + (warp * 8 + (lane & 7)) * L::kStgRow;
-#pragma unroll
-      for (int rnd = 0; rnd < 4; ++rnd) {
-        if ((lane >> 3) == rnd) {
-#pragma unroll
-          for (int x = 0; x < D / 2; x += 4)
-            *reinterpret_cast<uint4*>(slot + x * 4) = make_uint4(hv[x], hv[x + 1], hv[x + 2], hv[x + 3]);
-          if (e_cur >= 0) {
-            fence_proxy_async_smem();
-            bulk_store_s2g(a.part_o + (int64_t)e_cur * D, smem_u32(slot), D * 2);
-            bulk_commit();
-            bulk_wait_read_all();
-          }
-        }
-        __syncwarp();
-      }
-      e_cur = e_next;
-    }
-  } else if (warp == 8) {
-    // ========================================================= TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      uint32_t J = 0;
-      int64_t lo_next = __ldg(a.tile_bucket + first);
-      for (int n = 0; n < nitems && ok; ++n) {
-        const int64_t lo = lo_next;
-        if (n + 1 < nitems) lo_next = __ldg(a.tile_bucket + first + (n + 1) * stride);
-        const int32_t b = (int32_t)(lo % g.MB);
-        const int s = (int)((lo / g.MB) % g.num_seqs);
-        const int gk = (int)(lo / ((int64_t)g.MB * g.num_seqs));
-        const int32_t key0 = seq_start(g, s) + b * g.bs;
-        for (int j = 0; j < nchunks && ok; ++j, ++J) {
-          const int st = J & 1;
-          const uint32_t u = J >> 1;
-          const int tok = key0 + j * kBN;
-          if (u > 0) ok = mbar_wait(&bars[pKEmpty0 + st], (u - 1) & 1, g.err);
-          if (!ok) break;
-          mbar_expect_tx(&bars[pKFull0 + st], L::kTile);
-#pragma unroll
-          for (int hh = 0; hh < D / 64; ++hh)
-            tma_load_3d(smem + L::kK0 + st * L::kTile + hh * kRows * 128, &tmK, &bars[pKFull0 + st], hh * 64, gk, tok);
-          if (u > 0) ok = mbar_wait(&bars[pVEmpty0 + st], (u - 1) & 1, g.err);
-          if (!ok) break;
-          mbar_expect_tx(&bars[pVFull0 + st], L::kTile);
-#pragma unroll
-          for (int hh = 0; hh < D / 64; ++hh)
-            tma_load_3d(smem + L::kV0 + st * L::kTile + hh * kRows * 128, &tmV, &bars[pVFull0 + st], hh * 64, gk, tok);
-        }
-      }
-    }
-  } else if (warp == 9) {
-    // ========================================================= MMA issuer (whole warp)
-    constexpr uint32_t idS = idesc_bf16(kRows, kBN, false, false);
-    constexpr uint32_t idO = idesc_bf16(kRows, D, false, true);
-    const uint32_t sQ = smem_u32(smem + L::kQ);
-    const uint32_t sK0 = smem_u32(smem + L::kK0);
-    const uint32_t sV0 = smem_u32(smem + L::kV0);
-    auto issue_s = [&](int t, uint32_t jj) {
-      const uint32_t qb = sQ + t * L::kTile, kb = sK0 + (jj & 1) * L::kTile;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
-        mma_ss_lo(tmem + kColS + t * kBN, sdesc_lo(qb + off, 16), sdesc_lo(kb + off, 16), idS, kk > 0 ? 1u : 0u);
-      }
-      mma_commit_warp(&bars[pSFull0 + t]);
-    };
-    auto issue_pv = [&](int t, uint32_t jj, bool first_chunk) {
-      const uint32_t vb = sV0 + (jj & 1) * L::kTile;
-#pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk)
-        mma_ts_lo(tmem + kColO + t * 128, tmem + kColS + t * kBN + kColP + kk * 8, sdesc_lo(vb + kk * 2048, kRows * 128),
-                  idO, (!first_chunk || kk > 0) ? 1u : 0u);
-    };
-    uint32_t J = 0;
-    for (int n = 0; n < nitems && ok; ++n) {
-      ok = mbar_wait_warp(&bars[pQFull], n & 1, g.err) && mbar_wait_warp(&bars[pKFull0 + (J & 1)], (J >> 1) & 1, g.err);
-      if (!ok) break;
-      tc_fence_after();
-      issue_s(0, J);
-      issue_s(1, J);
-      mma_commit_warp(&bars[pKEmpty0 + (J & 1)]);
-      for (int j = 0; j < nchunks && ok; ++j) {
-        const uint32_t Jc = J + j;
-        const bool more = j + 1 < nchunks;
-        ok = mbar_wait_warp(&bars[pVFull0 + (Jc & 1)], (Jc >> 1) & 1, g.err) &&
-             mbar_wait_warp(&bars[pPFull0], Jc & 1, g.err);
-        if (ok && j == 0 && n > 0) ok = mbar_wait_warp(&bars[pODrained0], (n - 1) & 1, g.err);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(0, Jc, j == 0);
-        if (!more) mma_commit_warp(&bars[pOFull0]);
-        if (more) {
-          ok = mbar_wait_warp(&bars[pKFull0 + ((Jc + 1) & 1)], ((Jc + 1) >> 1) & 1, g.err);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(0, Jc + 1);
-        }
-        ok = mbar_wait_warp(&bars[pPFull1], Jc & 1, g.err);
-        if (ok && j == 0 && n > 0) ok = mbar_wait_warp(&bars[pODrained1], (n - 1) & 1, g.err);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, Jc, j == 0);
-        mma_commit_warp(&bars[pVEmpty0 + (Jc & 1)]);
-        if (!more) mma_commit_warp(&bars[pOFull1]);
-        if (more) {
-          issue_s(1, Jc + 1);
-          mma_commit_warp(&bars[pKEmpty0 + ((Jc + 1) & 1)]);
-        }
-      }
-      J += nchunks;
-    }
-    mma_commit_warp(&bars[pDone]);
-    mbar_wait_warp(&bars[pDone], 0, g.err);
-  }
-
-  // ------------------------------------------------------------- teardown
-  __syncthreads();
-  if (warp == 9) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
-}
-
-template <int D>
-cudaError_t launch_past_persistent(const Geom& g, const __nv_bfloat16* K, const __nv_bfloat16* V, const __nv_bfloat16* Q,
-                                   const Work& w, cudaStream_t st) {
-  CUtensorMap tk, tv;
-  cudaError_t e = make_rows_map(&tk, K, (uint64_t)g.T, g.Hkv, D, kBN);
-  if (e != cudaSuccess) return e;
-  e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kBN);
-  if (e != cudaSuccess) return e;
-  AttnArgs a{g, Q, nullptr, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, nullptr, nullptr, 0, 0,
-             nullptr, nullptr};
-  const int smem = PLayout<D>::kAlloc;
-  e = cudaFuncSetAttribute(attn_past_persistent_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, attn_past_persistent_kernel<D>);
-  if (e != cudaSuccess) return e;
-  if ((uint32_t)fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = past_tiles(g);
-  dim3 grid((unsigned)(tiles < nsm ? tiles : nsm));
-  attn_past_persistent_kernel<D><<<grid, kThreads, smem, st>>>(tk, tv, a);
-  return cudaGetLastError();
-}
-
 }  // namespace
-
-cudaError_t launch_attn_past(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
-                             const __nv_bfloat16* V, const Work& w, cudaStream_t st) {
-  if (g.T == 0 || g.k < 2 || g.R == 0) return cudaSuccess;
-  if (g.D == 64) return launch_past_persistent<64>(g, K, V, Q, w, st);
-  return launch_past_persistent<128>(g, K, V, Q, w, st);
-}
 
 namespace {
 // Grid of the own-block and naive modes: tile pairs (two heads of a group, or two
