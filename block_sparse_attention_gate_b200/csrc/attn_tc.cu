@@ -80,9 +80,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int per_blk = g.bs / kRows;
     s = blockIdx.y;
     const int32_t ts = seq_start(g, s), te = seq_end(g, s);
-    // The longest tiles start first.  Own mode: a tile's work grows with its place in the
-    // block, so the grid runs the blocks' last tiles first, then the ones before them.
-    // Naive mode: the work grows with the block index, so the grid runs backwards.
+    // Own mode: the tiles of a block run together, so its K/V chunks are shared through L2
+    // (the GPU runs under its power cap, and DRAM traffic saved there speeds up the other
+    // kernels), and inside a block the longest tiles (the last ones) start first.  Naive
+    // mode: the work grows with the block index, so the grid runs backwards.
     const int bx = kNaive ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
     if (a.own_head_pairs) {
       int qt;
@@ -90,8 +91,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         i_blk = bx / per_blk;
         qt = bx - i_blk * per_blk;
       } else {
-        qt = per_blk - 1 - bx / g.MB;
-        i_blk = bx - (per_blk - 1 - qt) * g.MB;
+        i_blk = bx / per_blk;
+        qt = per_blk - 1 - (bx - i_blk * per_blk);
       }
       const int32_t q0 = ts + i_blk * g.bs + qt * kRows;
       if (q0 >= te) return;
@@ -110,8 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         i_blk = bx / pairs;
         qp = bx - i_blk * pairs;
       } else {
-        qp = pairs - 1 - bx / g.MB;
-        i_blk = bx - (pairs - 1 - qp) * g.MB;
+        i_blk = bx / pairs;
+        qp = pairs - 1 - (bx - i_blk * pairs);
       }
       const int32_t q0 = ts + i_blk * g.bs + 2 * qp * kRows;
       if (q0 >= te) return;
