@@ -14,18 +14,22 @@
 //   decode_gate_kernel : one CTA per (sequence, KV head); the group's pooled keys are staged
 //                        in shared memory by 64-block chunks and one warp per query head
 //                        scores them, keeping per-lane top lists merged at the end.
-//   decode_attn_kernel : one CTA per (sequence, query head, selected block): eight warps
-//                        take rounds of 32 keys; a round loads 32 K rows coalesced (a lane
-//                        holds D/32 dimensions of each), forms the 32 dot products by a
-//                        butterfly reduce-scatter (lane j ends with key j's logit), runs
-//                        the online softmax, and accumulates P V with the lane again
-//                        holding D/32 dimensions.  The CTA's eight partial states are
-//                        combined into one normalised partial O and its LSE.
+//   decode_attn_tma_kernel: one CTA per (sequence, query head, selected block).  A producer
+//                        warp streams the block's keys and values by TMA, 128 keys per
+//                        stage, into a three-stage shared-memory ring; four consumer warps
+//                        each form 32 logits per stage (a lane per key, the key row read
+//                        from the swizzled stage, the query broadcast from shared memory),
+//                        run the online softmax and accumulate P V (a lane per D/32
+//                        dimensions).  The copies in flight, not the threads' registers,
+//                        carry the memory parallelism.  The four warps' states are combined
+//                        into one normalised partial O and its LSE.
 //   decode_merge_kernel: the top_k partials of a (sequence, head) merged by online softmax
 //                        into the final O (bf16) and LSE.
+#include <cudaTypedefs.h>
 #include <float.h>
 
 #include "moba_internal.cuh"
+#include "sm100.cuh"
 
 namespace moba {
 
@@ -33,7 +37,6 @@ namespace {
 
 constexpr int kGateChunk = 64;     // pooled-key rows staged per step of the gate
 constexpr int kGateWarps = 8;      // query heads scored at once per CTA
-constexpr int kAttnWarps = 8;
 constexpr float kLog2eD = 1.4426950408889634f;
 constexpr float kLn2D = 0.6931471805599453f;
 
@@ -123,147 +126,6 @@ __global__ void __launch_bounds__(kGateWarps * 32)
   }
 }
 
-// One (sequence, query head, selected block): normalised partial O (fp32) and its LSE.
-template <int D>
-__global__ void __launch_bounds__(kAttnWarps * 32)
-    decode_attn_kernel(Geom g, const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-                       const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ sel,
-                       float* __restrict__ part_o, float* __restrict__ part_lse) {
-  constexpr int kDL = D / 32;  // dimensions per lane
-  __shared__ float red_m[kAttnWarps], red_l[kAttnWarps];
-  __shared__ float red_o[kAttnWarps][D];
-  const int slot = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t unit = ((int64_t)s * g.Hq + h) * g.k + slot;
-  const int32_t b = __ldg(sel + unit);
-  if (b < 0) return;  // unused slot: the merge skips it
-  const int32_t ts = seq_start(g, s);
-  const int32_t len = seq_end(g, s) - ts;
-  const int32_t p = len - 1;
-  const int i = p / g.bs;
-  const int32_t t0 = ts + b * g.bs;
-  const int n = b == i ? p - b * g.bs + 1 : g.bs;  // own block: keys up to the new token
-  const int gk = h / g.G;
-  // this lane's query dimensions, pre-scaled into log2 units
-  float q[kDL];
-  {
-    const __nv_bfloat16* qp = Q + ((int64_t)s * g.Hq + h) * D + lane * kDL;
-#pragma unroll
-    for (int x = 0; x < kDL; ++x) q[x] = __bfloat162float(qp[x]) * g.scale_log2;
-  }
-  const int64_t kv_stride = (int64_t)g.Hkv * D;
-  const __nv_bfloat16* kbase = K + (int64_t)t0 * kv_stride + (int64_t)gk * D + lane * kDL;
-  const __nv_bfloat16* vbase = V + (int64_t)t0 * kv_stride + (int64_t)gk * D + lane * kDL;
-  float m = -INFINITY, l = 0.f;
-  float o[kDL];
-#pragma unroll
-  for (int x = 0; x < kDL; ++x) o[x] = 0.f;
-  for (int r0 = warp * 32; r0 < n; r0 += kAttnWarps * 32) {
-    const int nk = min(32, n - r0);
-    // partial dot products: v[j] = sum over this lane's dimensions of q . K[r0 + j]
-    float v[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      float acc = 0.f;
-      if (j < nk) {
-        const __nv_bfloat16* kp = kbase + (int64_t)(r0 + j) * kv_stride;
-        if constexpr (kDL == 4) {
-          const uint2 raw = __ldg(reinterpret_cast<const uint2*>(kp));
-          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-          const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
-          acc = fmaf(q[0], a.x, fmaf(q[1], a.y, fmaf(q[2], c.x, q[3] * c.y)));
-        } else {
-          const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(kp));
-          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw));
-          acc = fmaf(q[0], a.x, q[1] * a.y);
-        }
-      }
-      v[j] = acc;
-    }
-    // butterfly reduce-scatter: after step `off` a lane keeps the half of the entries whose
-    // index bit `off` equals its own lane bit; at the end lane j holds the sum for key j
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const bool upper = (lane & off) != 0;
-#pragma unroll
-      for (int x = 0; x < off; ++x) {
-        const float send = upper ? v[x] : v[x + off];
-        const float keep = upper ? v[x + off] : v[x];
-        v[x] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-      }
-    }
-    const float z = lane < nk ? v[0] : -INFINITY;  // logit of key r0 + lane, log2 units
-    float mx = z;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    const float m_new = fmaxf(m, mx);
-    const float alpha = exp2f(m - m_new);  // 0 on the first round (m = -inf)
-    const float pz = lane < nk ? exp2f(z - m_new) : 0.f;
-    float ps = pz;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-    l = l * alpha + ps;
-    m = m_new;
-#pragma unroll
-    for (int x = 0; x < kDL; ++x) o[x] *= alpha;
-    // the value rows of the round, eight at a time: the eight loads are in flight together
-    // (a loop, not unrolled, so the registers stay few and several CTAs fit on an SM)
-#pragma unroll 1
-    for (int j0 = 0; j0 < 32; j0 += 8) {
-      uint32_t vr[8][kDL / 2];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const __nv_bfloat16* vp = vbase + (int64_t)(r0 + j0 + j) * kv_stride;
-        if constexpr (kDL == 4) {
-          uint2 raw = make_uint2(0u, 0u);
-          if (j0 + j < nk) raw = __ldg(reinterpret_cast<const uint2*>(vp));
-          vr[j][0] = raw.x;
-          vr[j][1] = raw.y;
-        } else {
-          vr[j][0] = j0 + j < nk ? __ldg(reinterpret_cast<const uint32_t*>(vp)) : 0u;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float pj = __shfl_sync(0xffffffffu, pz, j0 + j);  // 0 for keys past the block's end
-#pragma unroll
-        for (int x = 0; x < kDL / 2; ++x) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vr[j][x]));
-          o[2 * x] = fmaf(pj, f.x, o[2 * x]);
-          o[2 * x + 1] = fmaf(pj, f.y, o[2 * x + 1]);
-        }
-      }
-    }
-  }
-  // combine the warps' states (a warp with no keys has m = -inf, l = 0, o = 0)
-  if (lane == 0) {
-    red_m[warp] = m;
-    red_l[warp] = l;
-  }
-#pragma unroll
-  for (int x = 0; x < kDL; ++x) red_o[warp][lane * kDL + x] = o[x];
-  __syncthreads();
-  if (warp == 0) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, red_m[w]);
-    float L = 0.f, acc[kDL];
-#pragma unroll
-    for (int x = 0; x < kDL; ++x) acc[x] = 0.f;
-#pragma unroll
-    for (int w = 0; w < kAttnWarps; ++w) {
-      const float sc = red_l[w] > 0.f ? exp2f(red_m[w] - M) : 0.f;
-      L += red_l[w] * sc;
-#pragma unroll
-      for (int x = 0; x < kDL; ++x) acc[x] = fmaf(red_o[w][lane * kDL + x], sc, acc[x]);
-    }
-    const float inv = 1.f / L;  // L >= 1: the maximum key contributes 2^0
-#pragma unroll
-    for (int x = 0; x < kDL; ++x) part_o[unit * D + lane * kDL + x] = acc[x] * inv;
-    if (lane == 0) part_lse[unit] = (M + log2f(L)) * kLn2D;
-  }
-}
-
 // The top_k partials of one (sequence, query head) merged by online softmax.
 template <int D>
 __global__ void __launch_bounds__(128)
@@ -297,6 +159,187 @@ __global__ void __launch_bounds__(128)
   if (lane == 0) LSE[row] = (M + log2f(L)) * kLn2D;
 }
 
+// One (sequence, query head, selected block) per CTA, fed by TMA: warp 4 streams the
+// block's keys and values, 128 keys per stage, into a three-stage shared-memory ring
+// (three 64 KB stages in flight per SM: the copies, not the threads' registers, hold the
+// memory parallelism), and warps 0-3 each take 32 keys of every stage.  A warp forms its
+// 32 logits with a lane per key (the key row read from the 128-byte-swizzled stage, the
+// query broadcast from shared memory), runs the online softmax over them, and accumulates
+// P V with a lane per D/32 dimensions.  The four warps' states are combined at the end into
+// the unit's normalised partial O and its LSE.
+constexpr int kTKeys = 128;     // keys per stage
+constexpr int kTStages = 3;
+constexpr int kTConsumers = 4;  // consumer warps (32 keys of each stage each)
+
+template <int D>
+struct DLayout {
+  static constexpr int kTile = kTKeys * D * 2;       // [128 x D] bf16
+  static constexpr int kK0 = 0;                       // kTStages stages
+  static constexpr int kV0 = kK0 + kTStages * kTile;  // kTStages stages
+  static constexpr int kQ = kV0 + kTStages * kTile;   // [D] fp32, pre-scaled
+  static constexpr int kRed = kQ + D * 4;             // [4][D] partial O + [4] m, l
+  static constexpr int kBar = kRed + kTConsumers * D * 4 + 2 * kTConsumers * 4;
+  static constexpr int kBytes = kBar + 64;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__((kTConsumers + 1) * 32, 1)
+    decode_attn_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                           Geom g, const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ sel,
+                           float* __restrict__ part_o, float* __restrict__ part_lse) {
+  using L = DLayout<D>;
+  constexpr int kDL = D / 32;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* empty = full + kTStages;
+  float* qs = reinterpret_cast<float*>(smem + L::kQ);
+  float* red_o = reinterpret_cast<float*>(smem + L::kRed);
+  float* red_m = red_o + kTConsumers * D;
+  float* red_l = red_m + kTConsumers;
+  const int slot = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t unit = ((int64_t)s * g.Hq + h) * g.k + slot;
+  const int32_t b = __ldg(sel + unit);
+  if (b < 0) return;  // unused slot: the merge skips it
+  const int32_t ts = seq_start(g, s);
+  const int32_t p = seq_end(g, s) - ts - 1;
+  const int i = p / g.bs;
+  const int32_t t0 = ts + b * g.bs;
+  const int n = b == i ? p - b * g.bs + 1 : g.bs;  // own block: keys up to the new token
+  const int nch = (n + kTKeys - 1) / kTKeys;
+  const int gk = h / g.G;
+  if (threadIdx.x < D) qs[threadIdx.x] = __bfloat162float(Q[((int64_t)s * g.Hq + h) * D + threadIdx.x]) * g.scale_log2;
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < kTStages; ++q) {
+      mbar_init(&full[q], 1);
+      mbar_init(&empty[q], kTConsumers);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  bool ok = true;
+  if (warp == kTConsumers) {
+    // ========================================================= TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      for (int c = 0; c < nch && ok; ++c) {
+        const int st = c % kTStages, u = c / kTStages;
+        if (u > 0) ok = mbar_wait(&empty[st], (u - 1) & 1, g.err);
+        if (!ok) break;
+        mbar_expect_tx(&full[st], 2 * L::kTile);
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh) {
+          tma_load_3d(smem + L::kK0 + st * L::kTile + hh * kTKeys * 128, &tmK, &full[st], hh * 64, gk, t0 + c * kTKeys);
+          tma_load_3d(smem + L::kV0 + st * L::kTile + hh * kTKeys * 128, &tmV, &full[st], hh * 64, gk, t0 + c * kTKeys);
+        }
+      }
+    }
+  } else {
+    // ========================================================= consumers
+    float m = -INFINITY, l = 0.f;
+    float o[kDL];
+#pragma unroll
+    for (int x = 0; x < kDL; ++x) o[x] = 0.f;
+    const int r = warp * 32 + lane;  // this lane's key row inside a stage (logits)
+    for (int c = 0; c < nch && ok; ++c) {
+      const int st = c % kTStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[st], (c / kTStages) & 1, g.err));
+      if (!ok) break;
+      const uint8_t* kst = smem + L::kK0 + st * L::kTile;
+      const uint8_t* vst = smem + L::kV0 + st * L::kTile;
+      // logit of key (c * 128 + r), log2 units: the row's 16-byte chunks sit at
+      // (chunk ^ (row & 7)) inside each 128-byte, 64-dimension atom
+      float z = 0.f;
+#pragma unroll
+      for (int a = 0; a < D / 64; ++a)
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 kv = *reinterpret_cast<const uint4*>(kst + a * kTKeys * 128 + r * 128 + ((ch ^ (r & 7)) << 4));
+          const float4 qa = *reinterpret_cast<const float4*>(qs + a * 64 + ch * 8);
+          const float4 qb = *reinterpret_cast<const float4*>(qs + a * 64 + ch * 8 + 4);
+          const float2 k0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kv.x));
+          const float2 k1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kv.y));
+          const float2 k2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kv.z));
+          const float2 k3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kv.w));
+          z = fmaf(qa.x, k0.x, fmaf(qa.y, k0.y, fmaf(qa.z, k1.x, fmaf(qa.w, k1.y, z))));
+          z = fmaf(qb.x, k2.x, fmaf(qb.y, k2.y, fmaf(qb.z, k3.x, fmaf(qb.w, k3.y, z))));
+        }
+      const bool live = c * kTKeys + r < n;
+      if (!live) z = -INFINITY;
+      float mx = z;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float m_new = fmaxf(m, mx);
+      if (m_new != -INFINITY) {  // warp-uniform: some key of this warp's share is live
+        const float alpha = exp2f(m - m_new);
+        const float pz = live ? exp2f(z - m_new) : 0.f;
+        float ps = pz;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+        l = l * alpha + ps;
+        m = m_new;
+#pragma unroll
+        for (int x = 0; x < kDL; ++x) o[x] *= alpha;
+        // P V: lane holds dimensions [kDL * lane, kDL * lane + kDL) of each value row
+        const int d0 = kDL * lane;
+        const int a = d0 >> 6, ch = (d0 & 63) >> 3, within = (d0 & 7) * 2;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+          const float pj = __shfl_sync(0xffffffffu, pz, j);
+          const int vr = warp * 32 + j;
+          const uint8_t* vp = vst + a * kTKeys * 128 + vr * 128 + ((ch ^ (vr & 7)) << 4) + within;
+          if constexpr (kDL == 4) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(vp);
+            const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+            const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+            o[0] = fmaf(pj, f0.x, o[0]);
+            o[1] = fmaf(pj, f0.y, o[1]);
+            o[2] = fmaf(pj, f1.x, o[2]);
+            o[3] = fmaf(pj, f1.y, o[3]);
+          } else {
+            const uint32_t raw = *reinterpret_cast<const uint32_t*>(vp);
+            const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw));
+            o[0] = fmaf(pj, f0.x, o[0]);
+            o[1] = fmaf(pj, f0.y, o[1]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);  // this warp's share of the stage is read
+    }
+    // combine the four warps' states (a warp without live keys has m = -inf, l = 0, o = 0)
+    if (lane == 0) {
+      red_m[warp] = m;
+      red_l[warp] = l;
+    }
+#pragma unroll
+    for (int x = 0; x < kDL; ++x) red_o[warp * D + lane * kDL + x] = o[x];
+  }
+  __syncthreads();
+  if (ok && warp == 0) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kTConsumers; ++w) M = fmaxf(M, red_m[w]);
+    float Lsum = 0.f, acc[kDL];
+#pragma unroll
+    for (int x = 0; x < kDL; ++x) acc[x] = 0.f;
+#pragma unroll
+    for (int w = 0; w < kTConsumers; ++w) {
+      const float sc = red_l[w] > 0.f ? exp2f(red_m[w] - M) : 0.f;
+      Lsum += red_l[w] * sc;
+#pragma unroll
+      for (int x = 0; x < kDL; ++x) acc[x] = fmaf(red_o[w * D + lane * kDL + x], sc, acc[x]);
+    }
+    const float inv = 1.f / Lsum;  // >= 1: the largest key contributes 2^0
+#pragma unroll
+    for (int x = 0; x < kDL; ++x) part_o[unit * D + lane * kDL + x] = acc[x] * inv;
+    if (lane == 0) part_lse[unit] = (M + log2f(Lsum)) * kLn2D;
+  }
+}
+
 template <int D>
 cudaError_t launch_decode_d(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                             const __nv_bfloat16* V, const float* Kbar, int32_t* sel, float* part_o,
@@ -309,10 +352,19 @@ cudaError_t launch_decode_d(const Geom& g, const __nv_bfloat16* Q, const __nv_bf
   else decode_gate_kernel<D, kMaxTopK - 1><<<ggrid, kGateWarps * 32, 0, st>>>(g, Q, Kbar, sel);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_attn_kernel<D><<<dim3((unsigned)g.k, (unsigned)g.Hq, (unsigned)g.num_seqs), kAttnWarps * 32, 0, st>>>(
-      g, Q, K, V, sel, part_o, part_lse);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  {
+    CUtensorMap tk, tv;
+    if ((e = make_rows_map(&tk, K, (uint64_t)g.T, g.Hkv, D, kTKeys)) != cudaSuccess) return e;
+    if ((e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kTKeys)) != cudaSuccess) return e;
+    const int smem = DLayout<D>::kAlloc;
+    if ((e = cudaFuncSetAttribute(decode_attn_tma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+      return e;
+    decode_attn_tma_kernel<D><<<dim3((unsigned)g.k, (unsigned)g.Hq, (unsigned)g.num_seqs), (kTConsumers + 1) * 32,
+                                smem, st>>>(tk, tv, g, Q, sel, part_o, part_lse);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const int64_t rows = (int64_t)g.num_seqs * g.Hq;
   decode_merge_kernel<D><<<(unsigned)((rows + 3) / 4), 128, 0, st>>>(g, sel, part_o, part_lse, O, LSE);
   return cudaGetLastError();
