@@ -1,4 +1,4 @@
-"""Pin of the attention kernels' FMA-pipe exp2 (``exp2_poly2`` in csrc/attn_tc.cu).
+"""Pin of the attention kernels' FMA-pipe exp2 (``exp2_poly2`` in csrc/attn_common.cuh).
 
 The kernel's exact fp32 operation sequence is replayed on the CPU with the constants read
 from the kernel source:
@@ -18,7 +18,7 @@ import re
 import numpy as np
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-KERNEL = os.path.join(ROOT, "block_sparse_attention_gate_b200", "csrc", "attn_tc.cu")
+KERNEL = os.path.join(ROOT, "block_sparse_attention_gate_b200", "csrc", "attn_common.cuh")
 REL_BOUND = 7.5e-5   # the bound the kernel's comment states
 
 
