@@ -1,4 +1,4 @@
-// Definitions shared by the tensor-core attention kernels (attn_tc.cu: own block + merge and
+// Definitions shared by the tensor-core attention kernels (attn_own.cu: own block + merge and
 // the mask-based form; attn_past.cu: past blocks): warp roles and the register split, the
 // tile and TMEM geometry, the FMA-pipe exp2, the kernels' argument block and the warp-wide
 // MMA issue with 32-bit descriptor words.
@@ -15,7 +15,8 @@ namespace moba {
 
 namespace {
 
-constexpr int kThreads = 384;  // warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA, 10-11 idle
+// Past-block kernel: warps 0-3 softmax tile 0, 4-7 softmax tile 1, 8 TMA, 9 MMA, 10-11 idle.
+constexpr int kThreads = 384;
 // Register split (setmaxnreg): the kernel is compiled for kLaunchRegs per thread; the third
 // warpgroup gives registers back so the two softmax warpgroups can hold a full S row.
 // 2 * 128 * kSoftmaxRegs + 128 * kOtherRegs must not exceed 384 * kLaunchRegs (checked on
@@ -24,9 +25,9 @@ constexpr uint32_t kLaunchRegs = 168;
 constexpr uint32_t kSoftmaxRegs = 216;
 constexpr uint32_t kOtherRegs = 72;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= 384 * kLaunchRegs, "register split too large");
-constexpr int kRows = 128;     // query rows per tile (M); two tiles per CTA
+constexpr int kRows = 128;     // query rows per tile (M)
 constexpr int kBN = 128;       // keys per chunk (N of S, K of PV)
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 512;  // past-block kernel: S and O of two tiles
 constexpr uint32_t kColS = 0;      // S of tile t at kColS + 128 t
 constexpr uint32_t kColP = 0;      // P of tile t (bf16 pairs) aliased at S + 0 .. S + 63
 constexpr uint32_t kColO = 256;    // O of tile t at kColO + 128 t
@@ -67,7 +68,6 @@ struct AttnArgs {
   float* part_lse;
   __nv_bfloat16* O;
   float* LSE;
-  int own_head_pairs;  // own mode: tiles are heads (2p, 2p+1) of one group (else query tiles 2p, 2p+1)
   int premerged;       // own mode: rows with two or more past partials have them folded in mo/mlse
   const __half* mo;    // [T * Hq, D] folded partial of each such row
   const float* mlse;   // [T * Hq] its LSE

@@ -352,7 +352,7 @@ cudaError_t launch_past_persistent(const Geom& g, const __nv_bfloat16* K, const 
   if (e != cudaSuccess) return e;
   e = make_rows_map(&tv, V, (uint64_t)g.T, g.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
-  AttnArgs a{g, Q, nullptr, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, nullptr, nullptr, 0, 0,
+  AttnArgs a{g, Q, nullptr, w.tile_off, w.tile_bucket, w.rows, w.part_o, w.part_lse, nullptr, nullptr, 0,
              nullptr, nullptr};
   const int smem = PLayout<D>::kAlloc;
   e = cudaFuncSetAttribute(attn_past_persistent_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -133,6 +133,7 @@ size_t carve(const moba::Geom& g, char* base, moba::Work* w) {
   x.sel = (int32_t*)take(sizeof(int32_t) * (size_t)g.T * g.Hq * g.k);
   x.kbar_hi = (__nv_bfloat16*)take(2 * (size_t)g.num_seqs * g.MB * g.Hkv * g.D);
   x.kbar_lo = (__nv_bfloat16*)take(2 * (size_t)g.num_seqs * g.MB * g.Hkv * g.D);
+  x.kbar_n2 = (float*)take(sizeof(float) * (size_t)g.num_seqs * g.MB * g.Hkv);
   x.bytes = off;
   if (w) *w = x;
   return off;
@@ -705,9 +706,12 @@ moba_status moba_read_device_error(int32_t* value, int clear) {
 
 namespace {
 constexpr size_t kNoAllocMaxKbarElems = (size_t)1 << 21;  // hi + lo: 2 x 2^21 bf16 = 8 MiB
+// Squared norms, one fp32 per pooled-key row (head_dim >= 64: at most 2^15 rows), stored
+// after hi and lo as pairs of bf16 slots.
+constexpr size_t kNoAllocNormSlots = 2 * (kNoAllocMaxKbarElems / 64);
 }  // namespace
 
-static __device__ __align__(256) __nv_bfloat16 g_gate_scratch[2 * kNoAllocMaxKbarElems];
+static __device__ __align__(256) __nv_bfloat16 g_gate_scratch[2 * kNoAllocMaxKbarElems + kNoAllocNormSlots];
 
 namespace {
 SymbolAddress g_gate_scratch_addr;
@@ -750,6 +754,7 @@ moba_status moba_gate_topk_noalloc(const moba_params* p, const void* Q, const fl
   moba::Work w{};
   w.kbar_hi = scratch;
   w.kbar_lo = scratch + kNoAllocMaxKbarElems;
+  w.kbar_n2 = reinterpret_cast<float*>(scratch + 2 * kNoAllocMaxKbarElems);
   cudaError_t e = moba::launch_gate(g, (const __nv_bfloat16*)Q, Kbar, sel, w, (cudaStream_t)stream);
   return e == cudaSuccess ? MOBA_OK : cuda_fail(e, "gate launch");
 }

@@ -74,6 +74,7 @@ struct Work {
   float* kbar;        // [num_seqs, MB, Hkv, D] (used by moba_fwd when the caller passes none)
   __nv_bfloat16* kbar_hi;  // [num_seqs, MB, Hkv, D] bf16 rn(Kbar) for the tensor-core gate
   __nv_bfloat16* kbar_lo;  // [num_seqs, MB, Hkv, D] bf16 rn(Kbar - hi)
+  float* kbar_n2;     // [num_seqs, Hkv, MB] squared norms of the pooled keys (gate score bound)
   int32_t* sel;       // [T, Hq, k] (used by moba_fwd when the caller passes none)
   size_t bytes;       // total
 };
@@ -96,6 +97,14 @@ cudaError_t launch_attn_past(const Geom& g, const __nv_bfloat16* Q, const __nv_b
 cudaError_t launch_attn_self(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                              const __nv_bfloat16* V, const int32_t* sel, const Work& w,
                              __nv_bfloat16* O, float* LSE, cudaStream_t st);
+// Own-block attention + merge (attn_own.cu): one 128-token tile of one head per CTA; rows
+// with two or more past partials read them folded from w.merged_* when premerged is set.
+cudaError_t launch_own_tiles(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                             const __nv_bfloat16* V, const int32_t* sel, const Work& w,
+                             __nv_bfloat16* O, float* LSE, int premerged, cudaStream_t st);
+cudaError_t launch_naive_tiles(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                               const __nv_bfloat16* V, const int32_t* sel, __nv_bfloat16* O, float* LSE,
+                               cudaStream_t st);
 // Mask-based form: every causal key scored, keys outside the selected blocks masked.
 cudaError_t launch_attn_naive(const Geom& g, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                               const __nv_bfloat16* V, const int32_t* sel, __nv_bfloat16* O, float* LSE,

@@ -97,6 +97,11 @@ MOBA_API moba_status moba_pool_keys(const moba_params* p, const void* K, float* 
  *         sel[..,1..m] = the m = min(top_k-1, i) past blocks with the largest
  *         <q, Kbar[b]>, by descending score, ties to the lower block index;
  *         remaining slots -1.
+ *         Resolution: scores are fp32 sums of q against Kbar split into bf16 hi + lo
+ *         (error up to 2^-18 B, B = |q| max_b |Kbar[b]| over the row's candidates).  With
+ *         top_k <= 5 the ranking compares the scores on a grid of step 2^-18 B / 0.49;
+ *         scores on the same grid point rank by block index.  Exact ties always go to
+ *         the lower block.
  *   workspace: >= moba_workspace_size(p) bytes, 256-byte aligned.
  */
 MOBA_API moba_status moba_gate_topk(const moba_params* p, const void* Q, const float* Kbar, int32_t* sel,
@@ -224,8 +229,9 @@ MOBA_API moba_status moba_pool_last_block(const moba_params* p, const void* K, f
  * while a CUDA graph is being captured (cudaMalloc is not allowed then), serving runtimes
  * that forbid allocation after start-up to keep memory use fixed, and host programs that
  * receive raw device pointers but no allocator.  The gate's scratch (the bf16 hi/lo split
- * of Kbar) lives in one device array of MOBA_NOALLOC_MAX_KBAR_ELEMS * 4 bytes (8 MiB) that
- * is compiled into the library; every GPU that loads the library holds it until exit.
+ * of Kbar and the pooled keys' squared norms) lives in one device array of
+ * MOBA_NOALLOC_MAX_KBAR_ELEMS * 4 bytes (8 MiB) plus 128 KiB that is compiled into the
+ * library; every GPU that loads the library holds it until exit.
  *  - Limit: num_seqs * ceil(max_seqlen / block_size) * num_kv_heads * head_dim must not
  *    exceed MOBA_NOALLOC_MAX_KBAR_ELEMS (2^21; a 1M-token sequence with 8 KV heads of
  *    dimension 128 at block size 2048 needs 2^19); larger problems get MOBA_ERR_UNSUPPORTED.
