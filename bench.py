@@ -154,11 +154,12 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def past_kernel_traffic(routed_rows: int):
-    """DRAM bytes per launch of the past-block attention kernel, from the committed ncu
-    record scaled by routed rows, or None when the kernel sources changed since the capture."""
+def kernel_traffic(record: str, units: int):
+    """DRAM bytes per launch of an attention kernel, from its committed ncu record (one
+    capture at 128K GQA) scaled by the units one launch processes, or None when the kernel's
+    sources changed since the capture."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "attn_past_traffic.json")
+    path = os.path.join(ROOT, "profiles", record)
     if not os.path.exists(path):
         return None, "no capture"
     with open(path) as f:
@@ -169,8 +170,8 @@ def past_kernel_traffic(routed_rows: int):
             h.update(f.read())
     if h.hexdigest() != rec["source_sha256"]:
         return None, "kernel changed since the capture"
-    per_row = (rec["dram_bytes_read"] + rec["dram_bytes_write"]) / rec["routed_rows"]
-    return per_row * routed_rows, "scaled from the %s capture by routed rows" % rec["workload"]
+    per_unit = (rec["dram_bytes_read"] + rec["dram_bytes_write"]) / rec["units"]
+    return per_unit * units, "scaled from the %s capture by %s" % (rec["workload"], rec["unit_kind"])
 
 
 def max_over_ranks(value: float, dist, device=None) -> float:
@@ -659,10 +660,13 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
         del staging, streams
         torch.cuda.empty_cache()
 
-    traffic, traffic_note = past_kernel_traffic(routed)
+    traffic, traffic_note = kernel_traffic("attn_past_traffic.json", routed)
+    own_traffic, own_note = kernel_traffic("attn_own_traffic.json", T * w.num_q_heads)
     peak_tf = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     past_s = stage_ms["past"] / 1e3
     achieved = fl["past"] / past_s / 1e12 if past_s > 0 else 0.0
+    own_s = stage_ms["own"] / 1e3
+    own_achieved = fl["own"] / own_s / 1e12 if own_s > 0 else 0.0
     eff_tf = (fl["attn"] + fl["gate"]) / (ms_step / 1e3) / 1e12
     res = {
         "metric": METRIC,
@@ -687,6 +691,11 @@ def run_ours(args, w: synth.Workload, rank: int, world: int, dist) -> dict | Non
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
                      "peak_kind": "%s bf16 sustained (kernel timed inside a long step)" % peak_kind,
                      "traffic": traffic, "traffic_note": traffic_note},
+        # the second attention kernel (own block + merge, with the partial pre-merge when used)
+        "roofline_own": {"bound": "tensor", "kernel": "own block + merge", "achieved": own_achieved,
+                         "peak": peak_tf, "unit": "TFLOP/s", "frac": own_achieved / peak_tf,
+                         "peak_kind": "%s bf16 sustained" % peak_kind,
+                         "traffic": own_traffic, "traffic_note": own_note},
         "clocks": clk,
         "gpu_launches": mb.moba_launches_per_forward(mp.p) * args.steps,
         "e2e": e2e,

@@ -151,6 +151,30 @@ __device__ __forceinline__ void mma_bf16_ts_warp(uint32_t d_tmem, uint32_t a_tme
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Warp-wide MMA issue with 32-bit descriptor words, for operands in the 128-byte-swizzled
+// K-major layout with 8-row groups 1024 bytes apart: such a descriptor (SBO 1024, version 1,
+// swizzle mode 2) has the constant upper word 0x40004040.
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 hi;\n\t.reg .b64 da, db;\n\t"
+      "mov.b32 hi, 0x40004040;\n\tmov.b64 da, {%1, hi};\n\tmov.b64 db, {%2, hi};\n\t"
+      "elect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 hi;\n\t.reg .b64 db;\n\t"
+      "mov.b32 hi, 0x40004040;\n\tmov.b64 db, {%2, hi};\n\t"
+      "elect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(acc)
+      : "memory");
+}
 // Arrive on an mbarrier once every tcgen05 operation issued so far by the elected lane completes.
 __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
   asm volatile(
