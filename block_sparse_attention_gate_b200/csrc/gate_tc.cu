@@ -19,7 +19,8 @@
 // this item or the next ones) are in flight while the current one is multiplied and scanned,
 // and the next item's Q tiles load as soon as the current item's MMAs are done.
 //
-// Selection cost.  With at most four blocks to choose (top_k <= 5) a score is not inserted
+// Selection cost.  With at most four blocks to choose (top_k <= 5) and more than one chunk of
+// candidates (the set-up below does not pay for itself on one chunk), a score is not inserted
 // into the running list one by one.  Each score becomes a key in [1, 2): the score scaled by
 // 0.49 / B, where B = |q| max_b |Kbar[b]| bounds every candidate's |s| (Cauchy-Schwarz), is
 // rounded onto the grid 2^-18 by one fma against 48 (whose ulp is 2^-18), moved to 1.5 + that
@@ -50,12 +51,14 @@ __device__ __forceinline__ bool ranks_before(float sa, int32_t ba, float sb, int
 // kMaxM: compile-time capacity (>= m), so the lists live in registers.  In a list the first
 // kMaxM - m slots hold sentinels that rank before every score and are never displaced, so
 // the m live slots are the last m and the current m-th best is always the last slot.
-template <int kMaxM>
+// kQuant: quantized keys + min/max network (kMaxM <= 4 only), else exact insertion.
+template <int kMaxM, bool kQuant_ = (kMaxM <= 4)>
 struct RowTopK {
-  static constexpr bool kQuant = kMaxM <= 4;  // quantized keys + min/max network
+  static constexpr bool kQuant = kQuant_;
+  static_assert(!kQuant || kMaxM <= 4, "the quantized form keeps at most four blocks");
   // the exact form keeps kLists lists; column x of a group goes to list x % kLists, so
   // kLists insertion chains run side by side
-  static constexpr int kLists = kQuant ? 1 : (kMaxM <= 8 ? 2 : 1);
+  static constexpr int kLists = kQuant ? 1 : (kMaxM <= 4 ? 4 : (kMaxM <= 8 ? 2 : 1));
   float ls[kLists][kMaxM];
   int32_t lb[kLists][kMaxM];
 
@@ -150,13 +153,18 @@ struct RowTopK {
         insert(ls[0], lb[0], __uint_as_float(bits & ~31u), b0 + 31 - (int32_t)(bits & 31u));
       }
     } else {
-      // Exact scores; a score at or below a list's last slot skips the insertion, and
-      // columns at or past the query block score -FLT_MAX, which never enters a list.
+      // Exact scores; columns at or past the query block score -FLT_MAX, which never enters
+      // a list.  Short lists take every score without a branch; longer ones skip a score at
+      // or below their last slot.
 #pragma unroll
       for (int x = 0; x < 32; ++x) {
         const int32_t b = b0 + x;
         const float sc = b < i ? __uint_as_float(v[x]) : -FLT_MAX;
-        if (sc > ls[x % kLists][kMaxM - 1]) insert(ls[x % kLists], lb[x % kLists], sc, b);
+        if constexpr (kMaxM <= 4) {
+          insert(ls[x % kLists], lb[x % kLists], sc, b);
+        } else {
+          if (sc > ls[x % kLists][kMaxM - 1]) insert(ls[x % kLists], lb[x % kLists], sc, b);
+        }
       }
     }
   }
@@ -335,34 +343,46 @@ __global__ void __launch_bounds__(kThreads, 3)
     // ========================================================= epilogue: running top-m
     const int r = tid;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    float scl = 0.f;
-    if constexpr (RowTopK<kMaxM>::kQuant) {
-      // the candidates' largest squared norm, by all 128 threads
-      const float* kn = kn2 + ((int64_t)s * g.Hkv + gk) * g.MB;
-      float kmax = 0.f;
-      for (int b = r; b < i; b += kRows) kmax = fmaxf(kmax, kn[b]);
+    // One selection form for the whole row: scan(tk, scl) walks the chunks.
+    auto select = [&](auto& tk, float scl) {
+      tk.init(m);
+      for (int c = 0; c < nch && ok; ++c) {
+        const int buf = c & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kTFull0 + buf], (c >> 1) & 1, g.err));
+        if (!ok) break;
+        tc_fence_after();
+        const int c0 = c * kCand;
+        scan_tmem(tmem + lane_off + buf * kCand, (min(kCand, i - c0) + 31) / 32,
+                  [&](const uint32_t (&v)[32], int gi) { tk.scan(v, c0 + gi * 32, i, scl); });
+        tc_fence_before();
+        mbar_arrive(&bars[kTFree0 + buf]);
+      }
+      if (ok && r < nrows) tk.write(sel + ((int64_t)(q0 + r) * g.Hq + h) * g.k, i, m, g.k);
+    };
+    // Quantized keys pay a per-row set-up (the key scale) that a single chunk of candidates
+    // does not repay: rows with at most kCand candidates take the exact insertion.
+    bool quant = false;
+    if constexpr (kMaxM <= 4) quant = i > kCand;  // the same for the whole CTA
+    if (quant) {
+      if constexpr (kMaxM <= 4) {
+        // the candidates' largest squared norm, by all 128 threads
+        const float* kn = kn2 + ((int64_t)s * g.Hkv + gk) * g.MB;
+        float kmax = 0.f;
+        for (int b = r; b < i; b += kRows) kmax = fmaxf(kmax, kn[b]);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-      if (lane == 0) red[warp] = kmax;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      kmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull], 0, g.err));
-      if (ok) scl = key_scale<D>(smem + L::kQ, r, kmax);
+        for (int o = 16; o > 0; o >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+        if (lane == 0) red[warp] = kmax;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        kmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull], 0, g.err));
+        const float scl = ok ? key_scale<D>(smem + L::kQ, r, kmax) : 0.f;
+        RowTopK<kMaxM, true> tk;
+        select(tk, scl);
+      }
+    } else {
+      RowTopK<kMaxM, false> tk;
+      select(tk, 0.f);
     }
-    RowTopK<kMaxM> tk;
-    tk.init(m);
-    for (int c = 0; c < nch && ok; ++c) {
-      const int buf = c & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kTFull0 + buf], (c >> 1) & 1, g.err));
-      if (!ok) break;
-      tc_fence_after();
-      const int c0 = c * kCand;
-      scan_tmem(tmem + lane_off + buf * kCand, (min(kCand, i - c0) + 31) / 32,
-                [&](const uint32_t (&v)[32], int gi) { tk.scan(v, c0 + gi * 32, i, scl); });
-      tc_fence_before();
-      mbar_arrive(&bars[kTFree0 + buf]);
-    }
-    if (ok && r < nrows) tk.write(sel + ((int64_t)(q0 + r) * g.Hq + h) * g.k, i, m, g.k);
   } else {
     // ========================================================= TMA + MMA issuer (warp 4)
     // The whole warp runs this loop: lane 0 issues the TMA copies, one elected lane the MMAs.

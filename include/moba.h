@@ -99,9 +99,9 @@ MOBA_API moba_status moba_pool_keys(const moba_params* p, const void* K, float* 
  *         remaining slots -1.
  *         Resolution: scores are fp32 sums of q against Kbar split into bf16 hi + lo
  *         (error up to 2^-18 B, B = |q| max_b |Kbar[b]| over the row's candidates).  With
- *         top_k <= 5 the ranking compares the scores on a grid of step 2^-18 B / 0.49;
- *         scores on the same grid point rank by block index.  Exact ties always go to
- *         the lower block.
+ *         top_k <= 5 and more than 64 candidate blocks the ranking compares the scores on
+ *         a grid of step 2^-18 B / 0.49; scores on the same grid point rank by block
+ *         index.  Exact ties always go to the lower block.
  *   workspace: >= moba_workspace_size(p) bytes, 256-byte aligned.
  */
 MOBA_API moba_status moba_gate_topk(const moba_params* p, const void* Q, const float* Kbar, int32_t* sel,

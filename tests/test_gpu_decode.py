@@ -27,6 +27,10 @@ CASES = [
     synth.Workload("dec_top1", [5000, 300, 4097], 4, 4, 128, 512, 1, seed=65),
     # odd group size, block 8192
     synth.Workload("dec_g3_bs8192", [20000, 8192], 6, 2, 128, 8192, 2, seed=66),
+    # eight query heads on one KV head with planted relevance: up to eight heads choose the
+    # same block, which is read once for each run of four of them
+    synth.Workload("dec_mqa8", [5000, 20000, 777], 8, 1, 128, 512, 3, seed=67, rope_theta=500000.0,
+                   plant=0.5),
 ]
 
 
