@@ -51,6 +51,12 @@ SMALL = {
     "chunks_d64_k8": synth.Workload("chunks_d64_k8", [17000], 2, 1, 64, 128, 8, seed=24,
                                     rope_theta=500000.0, plant=0.5),
     "chunks_k16": synth.Workload("chunks_k16", [9000, 300], 2, 1, 128, 128, 16, seed=25),
+    # the gate's KV-group kernel (exact selection, query heads in groups of four): two head
+    # groups per KV head at head_dim 64 (top_k 9), and top_k 16 at head_dim 128, both over
+    # more than 64 candidate blocks (several chunks, staged across items)
+    "grp_g8_k9_d64": synth.Workload("grp_g8_k9_d64", [9500, 3000], 8, 1, 64, 128, 9, seed=26,
+                                    rope_theta=500000.0, plant=0.5),
+    "grp_g4_k16": synth.Workload("grp_g4_k16", [12000, 700], 4, 1, 128, 128, 16, seed=27),
     # many short sequences
     "many_seqs": synth.Workload("many_seqs", list(np.random.default_rng(17).integers(1, 300, 300)), 2, 1, 64,
                                 128, 3, seed=17),
