@@ -105,6 +105,20 @@ __global__ void __launch_bounds__(kOwnThreads, 2)
   bool folded = false;     // the row's partials come folded (one partial in mo/mlse)
   if (!kNaive && warp < 4 && tid < nrows) {
     const int64_t qrow = (int64_t)(q0 + tid) * g.Hq + h;
+    // The row's partial O rows are read after the setup below; their fetch into L2 starts
+    // now, before the selection is known (every slot's row exists; unused ones cost only L2).
+    {
+      const char* p0 = reinterpret_cast<const char*>(a.part_o + qrow * (g.k - 1) * D);
+      const int nq = a.premerged ? 1 : g.k - 1;
+      for (int q = 0; q < nq; ++q)
+#pragma unroll
+        for (int off = 0; off < D * 2; off += 128) prefetch_l2(p0 + q * D * 2 + off);
+      if (a.premerged) {
+        const char* m0 = reinterpret_cast<const char*>(a.mo + qrow * D);
+#pragma unroll
+        for (int off = 0; off < D * 2; off += 128) prefetch_l2(m0 + off);
+      }
+    }
     bool run = true;
 #pragma unroll
     for (int q = 0; q < kMaxTopK - 1; ++q) {
